@@ -1,0 +1,404 @@
+"""Pins for the CPU oracle: each check compares it with something other than
+itself -- the E4M3 format definition, torch's own float8 conversion (an
+independent library routine), closed forms, float64 brute force and
+invariants -- chosen so that a dropped term, a wrong sign, index or tie rule,
+or a transposed operand fails at least one of them.
+
+Sources: "How to Profile DeepSeek-V3 Inference Kernels Using Triton
+Autotuning" (block-wise activation quant; FP8 GEMM with per-block scaling,
+BLOCK_K = 128); "Size the per-tensor FP8 dynamic-quant amax grid to the
+input" (exact amax, scale = amax / 448, bitwise-identical bytes; strided
+inputs and NaN parity from the review); "The Surgical Precision Flip ..."
+(Assumptions and Their Validity: E4M3 is 1/4/3 bits and widens to bf16
+losslessly).
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_dynamic_quantization_b200 import inputs
+
+F8 = torch.float8_e4m3fn
+
+
+def torch_decode(codes: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(codes, dtype=np.uint8))
+    return t.view(F8).to(torch.float64).numpy()
+
+
+def torch_encode(v: np.ndarray) -> np.ndarray:
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+    return t.to(F8).view(torch.uint8).numpy()
+
+
+ALL_CODES = np.arange(256, dtype=np.uint8)
+FINITE = np.array([c for c in range(256) if (c & 0x7F) != 0x7F], dtype=np.uint8)
+
+
+# ------------------------------------------------------------------ decode
+def test_decode_enumerates_format(oracle_mod):
+    v = oracle_mod.e4m3_decode(ALL_CODES)
+    nan = np.isnan(v)
+    assert sorted(np.flatnonzero(nan).tolist()) == [0x7F, 0xFF]
+    fin = v[~nan]
+    assert fin.size == 254
+    assert np.unique(fin).size == 253                 # +0 and -0 coincide
+    assert fin.max() == 448.0 and fin.min() == -448.0
+    pos = fin[fin > 0]
+    assert pos.min() == 2.0 ** -9                      # smallest subnormal
+    assert oracle_mod.e4m3_decode(0x08) == 2.0 ** -6   # smallest normal
+    assert oracle_mod.e4m3_decode(0x38) == 1.0         # exponent bias 7
+    assert np.signbit(oracle_mod.e4m3_decode(0x80))
+    # sign bit is bit 7
+    np.testing.assert_array_equal(v[0x80:][~nan[0x80:]], -v[:0x80][~nan[:0x80]])
+
+
+def test_decode_matches_torch(oracle_mod):
+    ours = oracle_mod.e4m3_decode(ALL_CODES)
+    ref = torch_decode(ALL_CODES)
+    np.testing.assert_array_equal(np.isnan(ours), np.isnan(ref))
+    m = ~np.isnan(ref)
+    np.testing.assert_array_equal(ours[m], ref[m])
+    np.testing.assert_array_equal(np.signbit(ours[m]), np.signbit(ref[m]))
+
+
+def test_e4m3_widens_to_bf16_losslessly(oracle_mod):
+    v = oracle_mod.e4m3_decode(FINITE)
+    back = torch.from_numpy(v).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(back, v)
+
+
+# ------------------------------------------------------------------ encode
+def test_encode_inverts_decode(oracle_mod):
+    v = oracle_mod.e4m3_decode(FINITE).astype(np.float32)
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(v), FINITE)
+
+
+def test_encode_special_values(oracle_mod):
+    cases = [
+        (448.0, 0x7E), (449.0, 0x7E), (464.0, 0x7E), (1e30, 0x7E), (np.inf, 0x7E),
+        (-448.0, 0xFE), (-np.inf, 0xFE), (-1e30, 0xFE),
+        (0.0, 0x00), (-0.0, 0x80), (2.0 ** -10, 0x00), (-(2.0 ** -10), 0x80),
+        (1.5 * 2.0 ** -10, 0x01), (-(1e-30), 0x80), (2.0 ** -6, 0x08),
+        (1.0625, 0x38),      # tie between 1.0 and 1.125 -> even mantissa 0
+        (1.1875, 0x3A),      # tie between 1.125 and 1.25 -> even mantissa 2
+        (432.0, 0x7E),       # tie between 416 and 448 -> even mantissa 6
+        (float(np.float32(1.0625) + np.float32(2.0 ** -20)), 0x39),
+    ]
+    vals = np.array([c[0] for c in cases], dtype=np.float32)
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(vals),
+                                  np.array([c[1] for c in cases], dtype=np.uint8))
+    nan_codes = oracle_mod.e4m3_encode(np.array([np.nan, -np.nan], np.float32))
+    assert all((c & 0x7F) == 0x7F for c in nan_codes)
+
+
+def _check_range_vs_torch(oracle_mod, first, count, sign):
+    bits = (np.arange(first, first + count, dtype=np.uint64) | sign).astype(np.uint32)
+    ours = oracle_mod.e4m3_encode_range(int(bits[0]), count)
+    ref = torch_encode(bits.view(np.float32))
+    bad = np.flatnonzero(ours != ref)
+    assert bad.size == 0, (hex(int(bits[bad[0]])), ours[bad[0]], ref[bad[0]])
+
+
+@pytest.mark.slow
+def test_encode_exhaustive_vs_torch(oracle_mod):
+    """Every fp32 bit pattern with |v| <= 464, both signs, against torch's
+    float8_e4m3fn conversion (RNE; it agrees with saturation up to 464 and
+    returns NaN above, where ours saturates by definition)."""
+    limit = 0x43E80001                       # up to and including 464.0
+    chunk = 1 << 24
+    for sign in (0, 0x80000000):
+        for first in range(0, limit, chunk):
+            _check_range_vs_torch(oracle_mod, first, min(chunk, limit - first), sign)
+
+
+def test_encode_nearest_by_brute_force(oracle_mod):
+    """Nearest representable value, ties to the even code, by enumeration."""
+    mags = oracle_mod.e4m3_decode(np.arange(0, 0x7F, dtype=np.uint8))   # 127 magnitudes
+    g = np.random.default_rng(7)
+    mids = (mags[1:] + mags[:-1]) / 2.0
+    mids32 = mids.astype(np.float32)
+    assert np.all(mids32.astype(np.float64) == mids)                     # exact
+    around = np.concatenate([mids32, np.nextafter(mids32, np.float32(0)),
+                             np.nextafter(mids32, np.float32(np.inf))])
+    rand = (np.exp2(g.uniform(-14, 9, 200000)) * g.uniform(1, 2, 200000)).astype(np.float32)
+    v = np.concatenate([around, rand, mags.astype(np.float32)])
+    v = v[v < 448]
+    d = np.abs(v.astype(np.float64)[:, None] - mags[None, :])
+    best = d.min(axis=1, keepdims=True)
+    cand = d == best
+    idx = np.where(cand.sum(1) == 2,
+                   np.argmax(cand & (np.arange(127) % 2 == 0)[None, :], axis=1),
+                   np.argmax(cand, axis=1))
+    expect = idx.astype(np.uint8)        # code == index for magnitudes 0x00..0x7E
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(v), expect)
+    np.testing.assert_array_equal(oracle_mod.e4m3_encode(-v), expect | 0x80)
+
+
+def test_encode_monotone(oracle_mod):
+    g = np.random.default_rng(3)
+    v = np.sort(np.concatenate([g.standard_normal(100000) * 100,
+                                g.standard_normal(10000) * 1e-2])).astype(np.float32)
+    dec = oracle_mod.e4m3_decode(oracle_mod.e4m3_encode(v))
+    assert np.all(np.diff(dec) >= 0)
+
+
+# ------------------------------------------------------------------ scale
+def test_scale_closed_form(oracle_mod):
+    assert oracle_mod.scale_from_amax(448.0) == 1.0
+    for k in range(-20, 21):
+        assert oracle_mod.scale_from_amax(448.0 * 2.0 ** k) == np.float32(2.0 ** k)
+    assert oracle_mod.scale_from_amax(0.0) == 0.0
+    assert np.isnan(oracle_mod.scale_from_amax(np.nan))
+    g = np.random.default_rng(11)
+    a = (np.exp2(g.uniform(-30, 30, 1000))).astype(np.float32)
+    ours = np.array([oracle_mod.scale_from_amax(x) for x in a], dtype=np.float32)
+    ref = (torch.from_numpy(a) / torch.tensor(448.0, dtype=torch.float32)).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+# ------------------------------------------------------------------ per-tensor
+def torch_quant(xf32: torch.Tensor, s: float) -> np.ndarray:
+    """Codes by torch: IEEE fp32 division then torch's float8 conversion
+    (saturation applied first, since torch maps large values to NaN)."""
+    q = xf32 / torch.tensor(s, dtype=torch.float32)
+    q = torch.clamp(q, -448.0, 448.0)
+    return q.to(F8).view(torch.uint8).numpy()
+
+
+def test_per_tensor_unit_scale_is_plain_conversion(oracle_mod):
+    x = inputs.activations_per_tensor(64)
+    xf = x.float()
+    xf = xf / xf.abs().max() * 448.0          # amax becomes exactly 448
+    xb = xf.to(torch.bfloat16)
+    assert xb.float().abs().max().item() == 448.0
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(xb))
+    assert s == 1.0
+    np.testing.assert_array_equal(q, xb.float().to(F8).view(torch.uint8).numpy())
+
+
+@pytest.mark.parametrize("m", [1, 64, 256])
+def test_per_tensor_matches_torch(oracle_mod, m):
+    x = inputs.activations_per_tensor(m)
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
+    amax = x.float().abs().max()
+    assert s == (amax / torch.tensor(448.0)).item()
+    np.testing.assert_array_equal(q, torch_quant(x.float(), s))
+
+
+def test_per_tensor_zero_convention(oracle_mod):
+    x = torch.zeros(3, 256, dtype=torch.bfloat16)
+    x[1, 5] = -0.0
+    x[2, :] = -0.0
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
+    assert s == 0.0
+    expect = np.where(np.signbit(x.float().numpy()), 0x80, 0x00).astype(np.uint8)
+    np.testing.assert_array_equal(q, expect)
+
+
+def test_per_tensor_nan_and_inf(oracle_mod):
+    x = inputs.activations_per_tensor(4, k=256)
+    xn = x.clone()
+    xn[2, 17] = float("nan")
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(xn))
+    assert np.isnan(s)
+    assert np.all((q & 0x7F) == 0x7F)
+    xi = x.clone()
+    xi[1, 3] = float("inf")
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(xi))
+    assert np.isinf(s)
+    fin = np.isfinite(xi.float().numpy())
+    assert np.all((q[fin] & 0x7F) == 0)                 # x / inf = +-0
+    assert (q[1, 3] & 0x7F) == 0x7F                    # inf / inf = NaN
+
+
+def test_per_tensor_round_trip_bound(oracle_mod):
+    x = inputs.activations_per_tensor(256)
+    q, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
+    xv = x.float().numpy().astype(np.float64)
+    dq = oracle_mod.e4m3_decode(q) * float(s)
+    r = np.abs(xv / float(s))
+    e = np.floor(np.log2(np.maximum(r, 2.0 ** -6)))
+    half_ulp = np.ldexp(1.0, (e - 4).astype(np.int64))      # 1/2 * 2^(e-3)
+    slack = 2.0 * np.abs(xv) * 2.0 ** -23
+    assert np.all(np.abs(dq - xv) <= half_ulp * float(s) + slack)
+    i = np.unravel_index(np.argmax(np.abs(xv)), xv.shape)
+    assert abs(abs(dq[i]) - float(np.abs(xv).max())) <= float(s) * 16   # amax element ~ 448*s
+
+
+def test_per_tensor_permutation_invariant(oracle_mod):
+    x = inputs.activations_per_tensor(64)
+    _, s = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
+    perm = torch.randperm(x.numel(), generator=torch.Generator().manual_seed(5))
+    xp = x.reshape(-1)[perm].reshape(x.shape).contiguous()
+    qp, sp = oracle_mod.quant_per_tensor(inputs.bf16_bits(xp))
+    assert sp == s
+
+
+def test_per_tensor_strided_rows(oracle_mod):
+    big = inputs.activations_per_tensor(32, k=512)
+    view = big[:, :256]                                  # row stride 512
+    q1, s1 = oracle_mod.quant_per_tensor(inputs.bf16_bits(view))
+    q2, s2 = oracle_mod.quant_per_tensor(inputs.bf16_bits(view.contiguous()))
+    assert s1 == s2
+    np.testing.assert_array_equal(q1, q2)
+    assert s1 == (view.float().abs().max() / 448.0).item()
+
+
+# ------------------------------------------------------------------ groups
+def torch_group_quant(x: torch.Tensor, rows: int, cols: int):
+    """Block quant by torch ops: amax over (rows x cols) blocks, fp32
+    division by 448, torch's float8 conversion."""
+    xf = x.float()
+    M, K = xf.shape
+    Mp = -(-M // rows) * rows
+    pad = torch.zeros(Mp, K)
+    pad[:M] = xf.abs()
+    amax = pad.reshape(Mp // rows, rows, K // cols, cols).amax(dim=(1, 3))
+    s = amax / torch.tensor(448.0)
+    s_full = s.repeat_interleave(rows, 0)[:M].repeat_interleave(cols, 1)
+    safe = torch.where(s_full == 0, torch.ones_like(s_full), s_full)
+    q = torch.clamp(xf / safe, -448, 448).to(F8).view(torch.uint8)
+    zero_code = torch.where(torch.signbit(xf), 0x80, 0x00).to(torch.uint8)
+    q = torch.where(s_full == 0, zero_code, q)
+    return q.numpy(), s.numpy()
+
+
+@pytest.mark.parametrize("m,k", [(1, 7168), (32, 7168), (5, 256)])
+def test_group128_matches_torch(oracle_mod, m, k):
+    x = inputs.activations_group(m, k=k)
+    q, s = oracle_mod.quant_group128(inputs.bf16_bits(x))
+    qr, sr = torch_group_quant(x, 1, 128)
+    np.testing.assert_array_equal(s, sr)
+    np.testing.assert_array_equal(q, qr)
+
+
+def test_group128_zero_group(oracle_mod):
+    x = inputs.activations_per_tensor(64)          # row 32 holds one zero group
+    q, s = oracle_mod.quant_group128(inputs.bf16_bits(x))
+    zr, zg = np.argwhere(s == 0)[0]
+    assert zr == 32
+    assert np.all(q[zr, 128 * zg:128 * zg + 128] == 0)
+    qr, sr = torch_group_quant(x, 1, 128)
+    np.testing.assert_array_equal(q, qr)
+    np.testing.assert_array_equal(s, sr)
+
+
+def test_group128_strided(oracle_mod):
+    big = inputs.activations_group(8, k=1024)
+    view = big[:, 128:640]
+    q1, s1 = oracle_mod.quant_group128(inputs.bf16_bits(view))
+    q2, s2 = oracle_mod.quant_group128(inputs.bf16_bits(view.contiguous()))
+    np.testing.assert_array_equal(q1, q2)
+    np.testing.assert_array_equal(s1, s2)
+
+
+@pytest.mark.parametrize("n", [256, 200])
+def test_block128_matches_torch(oracle_mod, n):
+    w = inputs.to_bf16(np.random.default_rng(n).standard_normal((n, 384)))
+    q, s = oracle_mod.quant_block128(inputs.bf16_bits(w))
+    qr, sr = torch_group_quant(w, 128, 128)
+    np.testing.assert_array_equal(s, sr)
+    np.testing.assert_array_equal(q, qr)
+
+
+# ------------------------------------------------------------------ GEMM
+def torch_block_gemm(qa, sa, qb, sb):
+    """float64 via torch: dequantised per-128 block products, scaled, summed."""
+    A = torch.from_numpy(torch_decode(qa))
+    B = torch.from_numpy(torch_decode(qb))
+    M, K = A.shape
+    N = B.shape[0]
+    out = torch.zeros(M, N, dtype=torch.float64)
+    sbn = torch.from_numpy(sb.astype(np.float64)).repeat_interleave(128, 0)[:N]
+    for kb in range(K // 128):
+        p = A[:, kb * 128:(kb + 1) * 128] @ B[:, kb * 128:(kb + 1) * 128].T
+        out += torch.from_numpy(sa[:, kb].astype(np.float64))[:, None] * sbn[None, :, kb] * p
+    return out.numpy()
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 8, 128), (5, 7, 256), (8, 200, 384), (3, 130, 128)])
+def test_gemm_matches_float64_brute_force(oracle_mod, m, n, k):
+    qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m * 1000 + n)
+    R, T = oracle_mod.block_gemm(qa, sa, qb, sb)
+    ref = torch_block_gemm(qa, sa, qb, sb)
+    np.testing.assert_allclose(R, ref, rtol=1e-12, atol=1e-300)
+    assert np.all(T >= np.abs(R) * (1 - 1e-12))
+
+
+def test_gemm_exact_integer_case(oracle_mod):
+    """Unit scales and codes for {0, +-1, +-2}: an exact integer matmul."""
+    g = np.random.default_rng(2)
+    vals = np.array([0x00, 0x38, 0xB8, 0x40, 0xC0], dtype=np.uint8)   # 0, 1, -1, 2, -2
+    qa = vals[g.integers(0, 5, (9, 256))]
+    qb = vals[g.integers(0, 5, (300, 256))]
+    sa = np.ones((9, 2), np.float32)
+    sb = np.ones((3, 2), np.float32)
+    R, _ = oracle_mod.block_gemm(qa, sa, qb, sb)
+    ia = torch.from_numpy(torch_decode(qa)).to(torch.int64)
+    ib = torch.from_numpy(torch_decode(qb)).to(torch.int64)
+    np.testing.assert_array_equal(R, (ia @ ib.T).numpy().astype(np.float64))
+    bf = oracle_mod.f64_to_bf16(R)
+    ref = torch.from_numpy(R).to(torch.float32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(bf, ref)
+
+
+def test_gemm_single_block_and_linearity(oracle_mod):
+    qa, sa, qb, sb = inputs.gemm_operands(4, 256, 512, seed=9)
+    R, _ = oracle_mod.block_gemm(qa, sa, qb, sb)
+    j = 2
+    only = sa.copy()
+    only[:, [i for i in range(4) if i != j]] = 0
+    Rj, _ = oracle_mod.block_gemm(qa, only, qb, sb)
+    A = torch_decode(qa[:, 128 * j:128 * j + 128])
+    B = torch_decode(qb[:, 128 * j:128 * j + 128])
+    sbn = np.repeat(sb[:, j].astype(np.float64), 128)[:256]
+    np.testing.assert_allclose(Rj, sa[:, j, None].astype(np.float64) * sbn[None, :] * (A @ B.T),
+                               rtol=1e-14)
+    doubled = sa.copy()
+    doubled[:, j] *= 2
+    R2, _ = oracle_mod.block_gemm(qa, doubled, qb, sb)
+    np.testing.assert_allclose(R2 - R, Rj, rtol=1e-9, atol=1e-12 * np.abs(R).max())
+
+
+def test_gemm_scale_index_uses_row_block_of_b(oracle_mod):
+    """Rows n and n+128 of B use different sb rows; rows within a block share one."""
+    qa, sa, qb, sb = inputs.gemm_operands(2, 256, 128, seed=4)
+    qb[128:] = qb[:128]
+    sb2 = sb.copy()
+    sb2[1] = sb[0] * 4
+    R, _ = oracle_mod.block_gemm(qa, sa, qb, sb2)
+    np.testing.assert_allclose(R[:, 128:], 4 * R[:, :128], rtol=1e-14)
+
+
+def test_gemm_points_equal_full(oracle_mod):
+    qa, sa, qb, sb = inputs.gemm_operands(6, 300, 256, seed=1)
+    R, T = oracle_mod.block_gemm(qa, sa, qb, sb)
+    g = np.random.default_rng(0)
+    ms, ns = g.integers(0, 6, 50), g.integers(0, 300, 50)
+    Rp, Tp = oracle_mod.block_gemm_points(qa, sa, qb, sb, ms, ns)
+    np.testing.assert_array_equal(Rp, R[ms, ns])
+    np.testing.assert_array_equal(Tp, T[ms, ns])
+
+
+def test_gemm_strided_operands(oracle_mod):
+    qa, sa, qb, sb = inputs.gemm_operands(4, 64, 256, seed=3)
+    wide = np.zeros((64, 512), np.uint8)
+    wide[:, :256] = qb
+    R1, _ = oracle_mod.block_gemm(qa, sa, qb, sb)
+    R2, _ = oracle_mod.block_gemm(qa, sa, wide[:, :256], sb)
+    np.testing.assert_array_equal(R1, R2)
+
+
+def test_f64_to_bf16_matches_torch(oracle_mod):
+    g = np.random.default_rng(1)
+    v = np.concatenate([g.standard_normal(100000) * 10.0 ** g.integers(-40, 38, 100000),
+                        [0.0, -0.0, 1e-45, -1e-45, 3.4e38, -3.4e38]]).astype(np.float32)
+    ours = oracle_mod.f64_to_bf16(v.astype(np.float64))
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_tolerance_formula(oracle_mod):
+    tol = oracle_mod.gemm_tolerance(np.array([1.0, 1.5, -3.0, 0.0]), np.zeros(4))
+    np.testing.assert_array_equal(tol, [2 * 2.0 ** -7, 2 * 2.0 ** -7, 2 * 2.0 ** -6, 2 * 2.0 ** -133])
