@@ -1,0 +1,507 @@
+// C ABI of the fp8q library: argument checks, launch selection, launches.
+// Declarations and the full contract are in include/fp8q.h.
+#include "fp8q.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "fp8q_status.cuh"
+#include "gemm_kernels.cuh"
+#include "quant_kernels.cuh"
+
+namespace fp8q {
+namespace {
+
+// ------------------------------------------------------------------ helpers
+bool log_enabled() {
+    static const bool on = [] {
+        const char* v = std::getenv("FP8Q_LOG");
+        return v && v[0] && v[0] != '0';
+    }();
+    return on;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
+
+struct DeviceInfo {
+    bool ready = false;
+    int status = FP8Q_OK;
+    int sms = 0;
+    int fused_capacity = 0;   // co-resident CTAs of the fused per-tensor kernel
+};
+
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+constexpr int kFusedU = 8;          // vectors per thread in the fused kernel
+constexpr int kStreamU = 4;         // vectors per thread per iteration elsewhere
+constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
+constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
+
+template <int BN, bool SWAP, int STAGES>
+cudaError_t set_gemm_smem() {
+    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                int(GemmCfg<BN, SWAP, STAGES>::kSmemBytes));
+}
+
+// Device facts, queried once per device.  FP8Q_ERR_NO_DEVICE unless the
+// current device is an sm_100 part.
+int device_info(DeviceInfo** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FP8Q_ERR_NO_DEVICE;
+    }
+    DeviceInfo& d = g_dev[dev];
+    if (!d.ready) {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        if (!d.ready) {
+            cudaDeviceProp prop;
+            if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) {
+                cudaGetLastError();
+                return FP8Q_ERR_NO_DEVICE;
+            }
+            d.status = FP8Q_OK;
+            if (prop.major != 10) d.status = FP8Q_ERR_NO_DEVICE;
+            d.sms = prop.multiProcessorCount;
+            int per_sm = 0;
+            if (d.status == FP8Q_OK &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm, per_tensor_fused_kernel<kFusedU, true>, kQuantThreads, 0) != cudaSuccess)
+                d.status = FP8Q_ERR_CUDA;
+            int per_sm_nc = 0;
+            if (d.status == FP8Q_OK &&
+                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &per_sm_nc, per_tensor_fused_kernel<kFusedU, false>, kQuantThreads, 0) != cudaSuccess)
+                d.status = FP8Q_ERR_CUDA;
+            d.fused_capacity = std::min(per_sm, per_sm_nc) * d.sms;
+            if (d.status == FP8Q_OK) {
+                cudaError_t e = cudaSuccess;
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 6>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 6>();
+                if (e == cudaSuccess) e = set_gemm_smem<64, true, 6>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, true, 5>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 6>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 4>();
+                if (e != cudaSuccess) { cudaGetLastError(); d.status = FP8Q_ERR_CUDA; }
+            }
+            d.ready = true;
+        }
+    }
+    *out = &d;
+    return d.status;
+}
+
+std::atomic<unsigned long long> g_launches{0};
+
+// Status of the launches just enqueued; counts them when they succeeded.
+int launch_status(int n = 1) {
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return FP8Q_ERR_CUDA;
+    g_launches.fetch_add(static_cast<unsigned long long>(n), std::memory_order_relaxed);
+    return FP8Q_OK;
+}
+
+// Streaming grid: enough CTAs for the data, capped at kBlocksPerSm per SM.
+int stream_grid(int64_t nvec, int sms) {
+    const int64_t need = (nvec + int64_t(kQuantThreads) * kStreamU - 1) /
+                         (int64_t(kQuantThreads) * kStreamU);
+    const int64_t cap = std::min<int64_t>(int64_t(sms) * kBlocksPerSm, kMaxPartials);
+    return int(std::max<int64_t>(1, std::min(need, cap)));
+}
+
+// Checks shared by the bf16 -> code entry points.
+int check_bf16_matrix(const void* x, int64_t rows, int64_t cols, int64_t ldx,
+                      const uint8_t* q, int64_t ldq, int64_t col_multiple) {
+    if (rows < 0 || cols < 0) return FP8Q_ERR_INVALID_ARG;
+    if (cols % col_multiple) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (rows == 0 || cols == 0) return FP8Q_OK;
+    if (!x || !q) return FP8Q_ERR_INVALID_ARG;
+    if (ldx < cols || ldq < cols) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ldx * 2) % 16 || !aligned8(q) || ldq % 8) return FP8Q_ERR_MISALIGNED;
+    return FP8Q_OK;
+}
+
+// ------------------------------------------------------------------ GEMM plan
+enum Mode { kNormal = 0, kSwap = 1 };
+struct TableRow { int64_t m_lo, m_hi, n_lo, n_hi; int mode, bn, splits; };
+const TableRow kGemmTable[] = {
+#include "launch_table.inc"
+};
+
+struct GemmPlan {
+    bool swap;
+    int bn, stages, splits, tiles_p, tiles_q, units, grid;
+    int64_t ldw;
+    size_t ws_bytes;
+};
+
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
+    GemmPlan pl{};
+    const TableRow* row = &kGemmTable[0];
+    for (const TableRow& r : kGemmTable)
+        if (M >= r.m_lo && M <= r.m_hi && N >= r.n_lo && N <= r.n_hi) { row = &r; break; }
+    pl.swap = row->mode == kSwap;
+    pl.bn = row->bn;
+    pl.stages = pl.swap ? (pl.bn == 128 ? 5 : 6) : (pl.bn == 256 ? 4 : 6);
+    const int G = int(K / 128);
+    const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
+    pl.tiles_p = int((rows_p + 127) / 128);
+    pl.tiles_q = int((rows_q + pl.bn - 1) / pl.bn);
+    const int64_t tiles = int64_t(pl.tiles_p) * pl.tiles_q;
+    int splits = row->splits;
+    if (splits <= 0) {
+        splits = 1;
+        if (tiles < sms) splits = int(std::max<int64_t>(1, sms / tiles));
+        splits = std::min(splits, std::max(1, G / 2));   // at least 2 K blocks per split
+    }
+    splits = std::max(1, std::min(splits, G));
+    if (pl.swap) {   // the swapped kernel stages ceil(G/splits) x bn scales in shared memory
+        while (((G + splits - 1) / splits) * pl.bn > 8192) ++splits;
+    }
+    pl.splits = splits;
+    pl.units = int(tiles * splits);
+    pl.grid = std::max(1, std::min(pl.units, sms));
+    pl.ldw = (N + 7) / 8 * 8;
+    pl.ws_bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(pl.ldw) * sizeof(float) : 0;
+    return pl;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        cudaGetLastError();
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// 2-D map over an E4M3 [rows, K] matrix (row pitch ld bytes), box of
+// 128 K-bytes x box_rows rows, 128-byte swizzle, zero fill out of bounds.
+bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_t ld, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(ld)};
+    cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN, bool SWAP, int STAGES>
+void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& p, int grid,
+                 cudaStream_t st) {
+    using C = GemmCfg<BN, SWAP, STAGES>;
+    block_gemm_kernel<BN, SWAP, STAGES><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+}
+
+}  // namespace
+}  // namespace fp8q
+
+using namespace fp8q;
+
+// ====================================================================== ABI
+extern "C" {
+
+const char* fp8q_status_string(int status) {
+    switch (status) {
+        case FP8Q_OK: return "FP8Q_OK";
+        case FP8Q_ERR_INVALID_ARG: return "FP8Q_ERR_INVALID_ARG";
+        case FP8Q_ERR_UNSUPPORTED_SHAPE: return "FP8Q_ERR_UNSUPPORTED_SHAPE";
+        case FP8Q_ERR_MISALIGNED: return "FP8Q_ERR_MISALIGNED";
+        case FP8Q_ERR_WORKSPACE: return "FP8Q_ERR_WORKSPACE";
+        case FP8Q_ERR_CUDA: return "FP8Q_ERR_CUDA";
+        case FP8Q_ERR_TIMEOUT: return "FP8Q_ERR_TIMEOUT";
+        case FP8Q_ERR_NO_DEVICE: return "FP8Q_ERR_NO_DEVICE";
+        default: return "FP8Q_ERR_UNKNOWN";
+    }
+}
+
+int fp8q_abi_version(void) { return (1 << 16) | 0; }
+
+// ------------------------------------------------------------ per-tensor
+size_t fp8_act_quant_per_tensor_workspace_size(int64_t, int64_t) {
+    return size_t(2 + kMaxPartials) * sizeof(uint32_t);
+}
+
+size_t fp8_act_amax_workspace_size(int64_t, int64_t) {
+    return size_t(kMaxPartials) * sizeof(uint32_t);
+}
+
+int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                             int64_t ldq, float* scale, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+    int rc = check_bf16_matrix(x, M, K, ldx, q, ldq, 8);
+    if (rc != FP8Q_OK) return rc;
+    if (!scale) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(scale)) return FP8Q_ERR_MISALIGNED;
+    if (!workspace || workspace_bytes < fp8_act_quant_per_tensor_workspace_size(M, K))
+        return FP8Q_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d)) != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0 || K == 0)
+        return cudaMemsetAsync(scale, 0, sizeof(float), st) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+
+    const int64_t vpr = K / 8, nvec = M * vpr;
+    const bool contig = (ldx == K && ldq == K);
+    uint32_t* ws = static_cast<uint32_t*>(workspace);
+    const int64_t fused_grid = (nvec + int64_t(kQuantThreads) * kFusedU - 1) /
+                               (int64_t(kQuantThreads) * kFusedU);
+    if (fused_grid <= std::min<int64_t>(d->fused_capacity, kMaxPartials)) {
+        int64_t spin = int64_t(1) << 24;
+        void* args[] = {(void*)&x, (void*)&nvec, (void*)&vpr, (void*)&ldx, (void*)&q,
+                        (void*)&ldq, (void*)&scale, (void*)&ws, (void*)&spin};
+        const void* fn = contig ? (const void*)per_tensor_fused_kernel<kFusedU, true>
+                                : (const void*)per_tensor_fused_kernel<kFusedU, false>;
+        if (log_enabled())
+            std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: fused grid=%lld\n",
+                         (long long)M, (long long)K, (long long)fused_grid);
+        const cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(unsigned(fused_grid)),
+                                                          dim3(kQuantThreads), args, 0, st);
+        if (e != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
+        return launch_status(1);
+    }
+    const int grid = stream_grid(nvec, d->sms);
+    uint32_t* partials = ws + 2;
+    if (log_enabled())
+        std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: amax+apply grid=%d\n",
+                     (long long)M, (long long)K, grid);
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    if (contig) {
+        amax_partial_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+        apply_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials, grid,
+                                                                     q, ldq, scale);
+    } else {
+        amax_partial_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+        apply_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials, grid,
+                                                                      q, ldq, scale);
+    }
+    return launch_status(2);
+}
+
+int fp8_act_amax(const void* x, int64_t M, int64_t K, int64_t ldx, uint32_t* amax_bits,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+    if (M < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
+    if (K % 8) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (!amax_bits) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(amax_bits)) return FP8Q_ERR_MISALIGNED;
+    if (M > 0 && K > 0) {
+        if (!x || ldx < K) return FP8Q_ERR_INVALID_ARG;
+        if (!aligned16(x) || (ldx * 2) % 16) return FP8Q_ERR_MISALIGNED;
+    }
+    if (!workspace || workspace_bytes < fp8_act_amax_workspace_size(M, K)) return FP8Q_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (M == 0 || K == 0)
+        return cudaMemsetAsync(amax_bits, 0, 4, st) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+    const int64_t vpr = K / 8, nvec = M * vpr;
+    const int grid = stream_grid(nvec, d->sms);
+    uint32_t* partials = static_cast<uint32_t*>(workspace);
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    if (ldx == K)
+        amax_partial_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+    else
+        amax_partial_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+    // Fold the partials into one word: a single CTA over `grid` words.
+    reduce_partials_kernel<<<1, kQuantThreads, 0, st>>>(partials, grid, amax_bits);
+    return launch_status(2);
+}
+
+int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
+                        const uint32_t* amax_bits, uint8_t* q, int64_t ldq, float* scale,
+                        void* stream) {
+    int rc = check_bf16_matrix(x, M, K, ldx, q, ldq, 8);
+    if (rc != FP8Q_OK) return rc;
+    if (!amax_bits) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(amax_bits) || (scale && !aligned4(scale))) return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d)) != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t vpr = K / 8, nvec = M * vpr;
+    if (nvec == 0) {
+        if (scale) scale_only_kernel<<<1, 32, 0, st>>>(amax_bits, scale);
+        return launch_status();
+    }
+    const int grid = stream_grid(nvec, d->sms);
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    if (ldx == K && ldq == K)
+        apply_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+                                                                     q, ldq, scale);
+    else
+        apply_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+                                                                      q, ldq, scale);
+    return launch_status();
+}
+
+// ------------------------------------------------------------ group / block
+int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                           int64_t ldq, float* scales, void* stream) {
+    int rc = check_bf16_matrix(x, M, K, ldx, q, ldq, 128);
+    if (rc != FP8Q_OK) return rc;
+    if (M == 0 || K == 0) return FP8Q_OK;
+    if (!scales) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(scales)) return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d)) != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t G = K / 128, groups = M * G;
+    const int64_t need = (groups * 16 + int64_t(kQuantThreads) * kStreamU - 1) /
+                         (int64_t(kQuantThreads) * kStreamU);
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(d->sms) * kBlocksPerSm)));
+    if (log_enabled())
+        std::fprintf(stderr, "[fp8q] group128 M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    if (ldx == K && ldq == K)
+        group128_quant_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+    else
+        group128_quant_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+    return launch_status();
+}
+
+int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* qb,
+                              int64_t ldqb, float* sb, void* stream) {
+    int rc = check_bf16_matrix(w, N, K, ldw, qb, ldqb, 128);
+    if (rc != FP8Q_OK) return rc;
+    if (N == 0 || K == 0) return FP8Q_OK;
+    if (!sb) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(sb)) return FP8Q_ERR_MISALIGNED;
+    if ((N + 127) / 128 > 65535) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d)) != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int64_t G = K / 128;
+    dim3 grid(unsigned(G), unsigned((N + 127) / 128));
+    block128_quant_kernel<<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(w), N, ldw, qb,
+                                                          ldqb, sb, G);
+    return launch_status();
+}
+
+// ------------------------------------------------------------ GEMM
+size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != FP8Q_OK) return 0;
+    return plan_gemm(M, N, K, d->sms).ws_bytes;
+}
+
+int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
+                   const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
+    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (!qa || !sa || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+    if (lda < K || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned16(qa) || !aligned16(qb) || !aligned16(y) || lda % 16 || ldb % 16 || (ldy * 2) % 16 ||
+        !aligned4(sa) || !aligned4(sb))
+        return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (K == 0) {
+        // Empty sum: Y = 0.
+        return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
+                   ? FP8Q_OK : FP8Q_ERR_CUDA;
+    }
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms);
+    if (pl.ws_bytes > 0) {
+        if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
+        if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
+    }
+    CUtensorMap tp, tq;
+    const uint8_t* P = pl.swap ? qb : qa;
+    const uint8_t* Q = pl.swap ? qa : qb;
+    const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
+    const int64_t ld_p = pl.swap ? ldb : lda, ld_q = pl.swap ? lda : ldb;
+    if (!make_tmap(&tp, P, rows_p, K, ld_p, 128) || !make_tmap(&tq, Q, rows_q, K, ld_q, pl.bn))
+        return FP8Q_ERR_CUDA;
+    GemmParams p;
+    p.sa = sa;
+    p.sb = sb;
+    p.y = static_cast<uint16_t*>(y);
+    p.ws = static_cast<float*>(workspace);
+    p.ldy = ldy;
+    p.ldw = pl.ldw;
+    p.M = int(M);
+    p.N = int(N);
+    p.G = int(K / 128);
+    p.tiles_p = pl.tiles_p;
+    p.tiles_q = pl.tiles_q;
+    p.splits = pl.splits;
+    p.units = pl.units;
+    if (log_enabled())
+        std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
+                     (long long)M, (long long)N, (long long)K, pl.swap ? "swap" : "normal", pl.bn,
+                     pl.stages, pl.splits, pl.units, pl.grid);
+    if (pl.swap) {
+        switch (pl.bn) {
+            case 16: launch_gemm<16, true, 6>(tp, tq, p, pl.grid, st); break;
+            case 32: launch_gemm<32, true, 6>(tp, tq, p, pl.grid, st); break;
+            case 64: launch_gemm<64, true, 6>(tp, tq, p, pl.grid, st); break;
+            default: launch_gemm<128, true, 5>(tp, tq, p, pl.grid, st); break;
+        }
+    } else {
+        if (pl.bn == 256) launch_gemm<256, false, 4>(tp, tq, p, pl.grid, st);
+        else launch_gemm<128, false, 6>(tp, tq, p, pl.grid, st);
+    }
+    if ((rc = launch_status()) != FP8Q_OK) return rc;
+    if (pl.splits > 1) {
+        const int64_t total = M * ((N + 3) / 4);
+        const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
+        splitk_reduce_kernel<<<g, 256, 0, st>>>(p.ws, pl.splits, p.M, p.N, pl.ldw, p.y, ldy);
+        rc = launch_status();
+    }
+    return rc;
+}
+
+// ------------------------------------------------------------ status
+unsigned long long fp8q_launch_count(void) {
+    return g_launches.load(std::memory_order_relaxed);
+}
+
+int fp8q_device_status(int* status, int reset) {
+    if (!status) return FP8Q_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc != FP8Q_OK) return rc;
+    if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+    *status = v;
+    if (reset) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+    }
+    return FP8Q_OK;
+}
+
+}  // extern "C"

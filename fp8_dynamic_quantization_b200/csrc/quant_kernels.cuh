@@ -1,0 +1,269 @@
+// Quantisation kernels: bf16 -> E4M3 codes + fp32 scales (sm_100a).
+//
+// All of them are HBM-bound streaming kernels: 16-byte vector loads of 8
+// bf16 values, several loads in flight per thread, grids sized to the input
+// (never a fixed grid with idle blocks; compare "Size the per-tensor FP8
+// dynamic-quant amax grid to the input", Description: a fixed 1024-block
+// grid with a 1024-way atomic sets a data-independent floor).
+//
+//  group128_quant_kernel     one pass: amax of each 1x128 group, its scale,
+//                            codes ("How to Profile DeepSeek-V3 Inference
+//                            Kernels Using Triton Autotuning", Benchmarking
+//                            the Activation Quantization Kernel).
+//  amax_partial_kernel       per-tensor amax, one partial max per CTA.
+//  apply_kernel              per-tensor apply pass: reduces the partials
+//                            (or reads one amax word), computes the scale,
+//                            writes codes.  Walks the tensor backwards, so
+//                            the part of x the amax pass read last is still
+//                            in L2 when it is read again.
+//  per_tensor_fused_kernel   small tensors: one launch; values stay in
+//                            registers across a bounded grid barrier.
+//  block128_quant_kernel     128x128 weight blocks (offline step).
+#pragma once
+
+#include "fp8q_common.cuh"
+#include "fp8q_status.cuh"
+
+namespace fp8q {
+
+constexpr int kQuantThreads = 256;
+
+// Address of 16-byte vector `i` of a row-major [rows, vec_per_row*8] bf16
+// matrix with row stride ld (elements).  CONTIG: ld == row length.
+template <bool CONTIG>
+__device__ __forceinline__ int64_t vec_offset(int64_t i, int64_t vec_per_row, int64_t ld) {
+    if (CONTIG) return i * 8;
+    const int64_t r = i / vec_per_row;
+    return r * ld + (i - r * vec_per_row) * 8;
+}
+
+// ---------------------------------------------------------------------------
+// Per-1x128-group quantisation.  16 threads own one group (16 x 8 values);
+// each thread carries U groups per iteration so U loads are in flight.
+// ---------------------------------------------------------------------------
+template <int U, bool CONTIG>
+__global__ void __launch_bounds__(kQuantThreads)
+group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
+                      uint8_t* __restrict__ q, int64_t ldq,
+                      float* __restrict__ scales, int64_t groups, int64_t G) {
+    const int sub = threadIdx.x & 15;
+    const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 4;
+    const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 4;
+    // The two halves of a warp own groups 2w and 2w+1 (g_stride is even), so
+    // testing the even one keeps the loop warp-uniform for the shuffles.
+    for (int64_t g0 = g_first; (g0 & ~int64_t(1)) < groups; g0 += U * g_stride) {
+        uint4 v[U];
+        int64_t xo[U], qo[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t g = g0 + u * g_stride;
+            if (CONTIG) {
+                xo[u] = g * 128 + sub * 8;
+                qo[u] = xo[u];
+            } else {
+                const int64_t r = g / G, c = g - r * G;
+                xo[u] = r * ldx + c * 128 + sub * 8;
+                qo[u] = r * ldq + c * 128 + sub * 8;
+            }
+            v[u] = (g < groups) ? ld_stream16(x + xo[u]) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t g = g0 + u * g_stride;
+            uint32_t m = absmax8(v[u]);
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            const float s = scale_from_amax(amax_bits_to_f32(m));
+            if (g < groups) {
+                st_stream8(q + qo[u], quant8(v[u], s));
+                if (sub == 0) scales[g] = s;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per-tensor amax: partial max per CTA into partials[blockIdx.x].
+// ---------------------------------------------------------------------------
+template <int U, bool CONTIG>
+__global__ void __launch_bounds__(kQuantThreads)
+amax_partial_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
+                    int64_t ldx, uint32_t* __restrict__ partials) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
+    uint32_t m = 0;
+    for (int64_t i0 = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x; i0 < nvec; i0 += U * stride) {
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            v[u] = (i < nvec) ? ld_stream16(x + vec_offset<CONTIG>(i, vec_per_row, ldx))
+                              : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
+    }
+    m = block_max<kQuantThreads>(m, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = m;
+}
+
+// ---------------------------------------------------------------------------
+// Per-tensor apply: amax = max(partials[0:nparts]); scale; codes.
+// ---------------------------------------------------------------------------
+template <int U, bool CONTIG>
+__global__ void __launch_bounds__(kQuantThreads)
+apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, int64_t ldx,
+             const uint32_t* __restrict__ partials, int nparts,
+             uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale_out) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < nparts; i += kQuantThreads) m = max(m, __ldcg(partials + i));
+    m = block_max<kQuantThreads>(m, red);
+    const float s = scale_from_amax(amax_bits_to_f32(m));
+    if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = s;
+
+    const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
+    const int64_t span = U * stride;
+    const int64_t first = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
+    const int64_t iters = (nvec + span - 1) / span;
+    for (int64_t it = iters - 1; it >= 0; --it) {       // backwards: L2 hits first
+        const int64_t i0 = it * span + first;
+        uint4 v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            v[u] = (i < nvec) ? ld_stream16(x + vec_offset<CONTIG>(i, vec_per_row, ldx))
+                              : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t i = i0 + u * stride;
+            if (i < nvec) {
+                const int64_t qo = CONTIG ? i * 8 : vec_offset<false>(i, vec_per_row, ldq);
+                st_stream8(q + qo, quant8(v[u], s));
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Per-tensor, single launch, for tensors that fit in the registers of one
+// co-resident grid (cooperative launch).  Barrier state lives in the
+// caller's workspace: ws[0] arrival count, ws[1] generation, ws[2..] one
+// partial max per CTA.  The last CTA to arrive resets the count and bumps
+// the generation; the others wait for the generation to change, at most
+// `spin_limit` polls, after which they record FP8Q_ERR_TIMEOUT and return
+// without writing outputs.
+// ---------------------------------------------------------------------------
+template <int U, bool CONTIG>
+__global__ void __launch_bounds__(kQuantThreads)
+per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
+                        int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
+                        float* __restrict__ scale_out, uint32_t* ws, int64_t spin_limit) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    __shared__ int s_ok;
+    const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
+    const int64_t first = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
+    volatile uint32_t* vws = ws;
+    uint32_t gen0 = 0;
+    if (threadIdx.x == 0) gen0 = vws[1];
+
+    uint4 v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = first + u * stride;
+        v[u] = (i < nvec) ? ld_stream16(x + vec_offset<CONTIG>(i, vec_per_row, ldx))
+                          : make_uint4(0, 0, 0, 0);
+    }
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
+    m = block_max<kQuantThreads>(m, red);
+
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        ws[2 + blockIdx.x] = m;
+        __threadfence();
+        const uint32_t arrived = atomicAdd(ws, 1u);
+        if (arrived == gridDim.x - 1) {
+            ws[0] = 0;
+            __threadfence();
+            atomicAdd(ws + 1, 1u);
+        } else {
+            int64_t n = 0;
+            while (vws[1] == gen0) {
+                if (++n > spin_limit) { ok = 0; record_error(6 /* FP8Q_ERR_TIMEOUT */); break; }
+                __nanosleep(64);
+            }
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    if (!s_ok) return;
+
+    uint32_t mm = 0;
+    for (int i = threadIdx.x; i < int(gridDim.x); i += kQuantThreads) mm = max(mm, __ldcg(ws + 2 + i));
+    mm = block_max<kQuantThreads>(mm, red);
+    const float s = scale_from_amax(amax_bits_to_f32(mm));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+        const int64_t i = first + u * stride;
+        if (i < nvec) {
+            const int64_t qo = CONTIG ? i * 8 : vec_offset<false>(i, vec_per_row, ldq);
+            st_stream8(q + qo, quant8(v[u], s));
+        }
+    }
+}
+
+// out = max(partials[0:n]); one CTA.
+__global__ void __launch_bounds__(kQuantThreads)
+reduce_partials_kernel(const uint32_t* __restrict__ partials, int n, uint32_t* __restrict__ out) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < n; i += kQuantThreads) m = max(m, __ldcg(partials + i));
+    m = block_max<kQuantThreads>(m, red);
+    if (threadIdx.x == 0) *out = m;
+}
+
+// scale = amax / 448 from an amax word, for an empty apply.
+__global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float* __restrict__ scale) {
+    if (threadIdx.x == 0) *scale = scale_from_amax(amax_bits_to_f32(*amax_bits));
+}
+
+// ---------------------------------------------------------------------------
+// 128x128 block quantisation of a weight W[N,K]: one CTA per block; each
+// thread keeps its 8 vectors in registers between the amax and the apply.
+// grid = (K/128, ceil(N/128)).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQuantThreads)
+block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
+                      uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sb, int64_t G) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    const int64_t kb = blockIdx.x, nb = blockIdx.y;
+    uint4 v[8];
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int j = threadIdx.x + u * kQuantThreads;       // 0..2047
+        const int64_t r = nb * 128 + (j >> 4);
+        const int c = (j & 15) * 8;
+        v[u] = (r < N) ? ld_stream16(w + r * ldw + kb * 128 + c) : make_uint4(0, 0, 0, 0);
+        m = max(m, absmax8(v[u]));
+    }
+    m = block_max<kQuantThreads>(m, red);
+    const float s = scale_from_amax(amax_bits_to_f32(m));
+    if (threadIdx.x == 0) sb[nb * G + kb] = s;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int j = threadIdx.x + u * kQuantThreads;
+        const int64_t r = nb * 128 + (j >> 4);
+        const int c = (j & 15) * 8;
+        if (r < N) st_stream8(q + r * ldq + kb * 128 + c, quant8(v[u], s));
+    }
+}
+
+}  // namespace fp8q

@@ -1,0 +1,189 @@
+/*
+ * fp8q -- C ABI of the FP8 (E4M3) dynamic-quantisation linear path on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The path has two halves:
+ *   1. dynamic activation quantisation: an exact amax reduction (over the
+ *      whole tensor, or per 1x128 group along K), scale = fl32(amax / 448),
+ *      codes = e4m3_rne_sat(fl32(x / scale));
+ *   2. the block-scaled FP8 GEMM that consumes those codes: A scaled per
+ *      1x128 group, B per 128x128 block, fp32 accumulation, bf16 output.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [P1] "How to Profile DeepSeek-V3 Inference Kernels Using Triton
+ *        Autotuning": "Understanding the Autotuned Kernels in DeepSeek-V3"
+ *        (block-wise activation quantisation producing FP8 values and
+ *        per-block scales; FP8 GEMM with per-block scaling), "Benchmarking
+ *        the FP8 GEMM Kernel" (BLOCK_SIZE_K = 128; codes plus scale tensors
+ *        a_s, b_s), "Benchmarking the Activation Quantization Kernel"
+ *        (act_quant(x, block_size=128) returns codes and scales).
+ *   [P2] "Size the per-tensor FP8 dynamic-quant amax grid to the input"
+ *        (TensorRT-LLM pull request 16569): "Description" (per-tensor amax
+ *        with an input-sized grid, then an apply-only pass), "Test Coverage"
+ *        (amax is exact; scale = amax / 448; bitwise-identical bytes), the
+ *        review comments (strided 2-D inputs; NaN handling).
+ *
+ * Conventions shared by every entry point
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library allocates nothing per call; it enqueues work on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream) and returns
+ *     before the work completes.
+ *   - Matrices are row-major with unit inner stride; `ld*` is the row
+ *     stride in ELEMENTS (>= the row length).  bf16 tensors are passed as
+ *     `const void*` holding IEEE bfloat16 bit patterns; E4M3 codes as
+ *     uint8_t (OCP FP8 E4M3: 1 sign, 4 exponent, 3 mantissa bits, bias 7,
+ *     no infinity, NaN = 0x7F/0xFF, max finite 448).
+ *   - Alignment: bf16 matrices (inputs and the GEMM output) and the GEMM's
+ *     code operands must be 16-byte aligned with row pitches (ld * element
+ *     size) that are multiples of 16 bytes; code OUTPUTS of the quantisation
+ *     calls 8-byte aligned with row pitches that are multiples of 8 bytes;
+ *     scale pointers 4-byte aligned.  Otherwise FP8Q_ERR_MISALIGNED.
+ *   - Arguments are checked on the host before anything is enqueued; on
+ *     any error nothing is enqueued.  A failed launch returns FP8Q_ERR_CUDA.
+ *   - Zero convention: an all-zero tensor (per-tensor path) or group (group
+ *     and block paths) gets scale 0.0f and signed-zero codes (0x00, or 0x80
+ *     where x is -0).  The GEMM consumes a zero scale as a zero
+ *     contribution.
+ *   - NaN / Inf: amax propagates NaN (any NaN makes amax NaN), else Inf.
+ *     The scale is then non-finite and the codes are E4M3 of x / scale
+ *     (NaN codes, or signed zeros for finite x over an infinite scale).
+ *   - Determinism: the same inputs give the same bytes, whatever the
+ *     launch configuration chosen.
+ *   - Environment: FP8Q_LOG=1 prints the launch chosen for every call to
+ *     stderr.  No environment variable changes numerics.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Status codes returned (as int) by every call. */
+typedef enum fp8q_status {
+    FP8Q_OK = 0,
+    FP8Q_ERR_INVALID_ARG = 1,       /* null pointer, negative size, ld < row length */
+    FP8Q_ERR_UNSUPPORTED_SHAPE = 2, /* K not a multiple of the required width */
+    FP8Q_ERR_MISALIGNED = 3,        /* pointer or row pitch alignment violated */
+    FP8Q_ERR_WORKSPACE = 4,         /* workspace missing or too small */
+    FP8Q_ERR_CUDA = 5,              /* a CUDA runtime call or launch failed */
+    FP8Q_ERR_TIMEOUT = 6,           /* a bounded device-side wait gave up */
+    FP8Q_ERR_NO_DEVICE = 7          /* no usable sm_100 device */
+} fp8q_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fp8q_status_string(int status);
+
+/* ABI version of this header, (major << 16) | minor. */
+int fp8q_abi_version(void);
+
+/* ------------------------------------------------------------------ */
+/* Per-tensor dynamic quantisation  ([P2] Description, Test Coverage)  */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of device workspace fp8_act_quant_per_tensor needs for an [M,K]
+ * input on the current device.  The workspace must be ZERO-FILLED before
+ * its first use; every completed call leaves it ready for the next call.
+ * Calls sharing one workspace must be ordered (same stream, or joined).
+ * After FP8Q_ERR_TIMEOUT the caller must zero it again. */
+size_t fp8_act_quant_per_tensor_workspace_size(int64_t M, int64_t K);
+
+/* x: bf16 [M,K], row stride ldx.  Writes codes q: uint8 [M,K], row stride
+ * ldq, and *scale (one fp32 on the device) = fl32(amax / 448), with
+ * amax = max |x| over the whole tensor (exact).  K must be a multiple of 8.
+ * M == 0 or K == 0 writes scale 0 and nothing else.  Small tensors take a
+ * single launch with a bounded grid barrier; larger ones take an amax pass
+ * with an input-sized grid and then an apply pass. */
+int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx,
+                             uint8_t* q, int64_t ldq, float* scale,
+                             void* workspace, size_t workspace_bytes,
+                             void* stream);
+
+/* The two halves of the per-tensor path, for callers that combine the amax
+ * of several shards (e.g. a max all-reduce across ranks) before applying.
+ *
+ * fp8_act_amax: writes *amax_bits (one uint32 on the device) = the bf16 bit
+ * pattern of max |x| over x[M,K] (NaN > Inf > finite under unsigned order),
+ * so the max of several shards' words is the amax of their union.
+ * Workspace: fp8_act_amax_workspace_size(M, K) bytes; needs no zero fill. */
+size_t fp8_act_amax_workspace_size(int64_t M, int64_t K);
+int fp8_act_amax(const void* x, int64_t M, int64_t K, int64_t ldx,
+                 uint32_t* amax_bits, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* fp8_act_quant_apply: scale = fl32(amax / 448) from *amax_bits (device),
+ * written to *scale (device, may be NULL), and codes of x[M,K] into q. */
+int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
+                        const uint32_t* amax_bits, uint8_t* q, int64_t ldq,
+                        float* scale, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Per-1x128-group quantisation along K ([P1] act_quant, block 128)    */
+/* ------------------------------------------------------------------ */
+
+/* x: bf16 [M,K] (row stride ldx), K a multiple of 128.  Writes codes
+ * q: uint8 [M,K] (row stride ldq) and scales: fp32 [M, K/128] row-major
+ * contiguous, scales[m*(K/128)+g] = fl32(amax(x[m,128g:128g+128]) / 448).
+ * One pass over x; no workspace. */
+int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx,
+                           uint8_t* q, int64_t ldq, float* scales, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Per-128x128-block weight quantisation ([P1] b_s: one scale per      */
+/* 128x128 block of the weight).  Auxiliary (offline) step.            */
+/* ------------------------------------------------------------------ */
+
+/* w: bf16 [N,K] (row stride ldw), K a multiple of 128.  Writes codes
+ * qb: uint8 [N,K] (row stride ldqb) and sb: fp32 [ceil(N/128), K/128]
+ * row-major contiguous; the last row block may hold fewer than 128 rows. */
+int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw,
+                              uint8_t* qb, int64_t ldqb, float* sb, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Block-scaled FP8 GEMM ([P1] FP8 GEMM with per-block scaling,         */
+/* BLOCK_SIZE_K = 128)                                                  */
+/* ------------------------------------------------------------------ */
+
+/* Bytes of device workspace fp8_block_gemm needs for (M, N, K) on the
+ * current device (split-K partial sums for skinny M; 0 when unused).
+ * The workspace needs no zero fill. */
+size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* Y = A * B^T with block scales:
+ *   Y[m,n] = bf16_rne( sum_kb sa[m,kb] * sb[n/128,kb]
+ *                       * sum_{k in block kb} A[m,k] * B[n,k] )
+ * accumulated in fp32 (the per-block partial from the tensor cores is
+ * multiplied by sa*sb in fp32 registers and added to an fp32 sum).
+ *   qa: E4M3 [M,K], row stride lda        sa: fp32 [M, K/128] contiguous
+ *   qb: E4M3 [N,K], row stride ldb        sb: fp32 [ceil(N/128), K/128]
+ *   y : bf16 [M,N], row stride ldy
+ * K must be a multiple of 128; M, N >= 0 arbitrary (tails handled).
+ * The launch (tile shape, operand swap, split-K) is chosen per shape from
+ * a compiled table.  Bounded device waits report FP8Q_ERR_TIMEOUT through
+ * fp8q_device_status. */
+int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
+                   const uint8_t* qb, int64_t ldb, const float* sb,
+                   void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* Device status                                                       */
+/* ------------------------------------------------------------------ */
+
+/* Synchronises the current device and stores in *status the first error a
+ * kernel recorded since the last reset (FP8Q_OK if none; FP8Q_ERR_TIMEOUT
+ * when a bounded wait gave up).  reset != 0 clears it afterwards. */
+int fp8q_device_status(int* status, int reset);
+
+/* Number of kernels this library has launched in the process so far (all
+ * devices, all streams); a diagnostic for benchmarks. */
+unsigned long long fp8q_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -68,6 +68,7 @@ def _load():
         lib.oracle_amax.argtypes = [_p, _i64, _i64, _i64]
         lib.oracle_amax.restype = ctypes.c_float
         lib.oracle_quant_per_tensor.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
+        lib.oracle_quant_apply.argtypes = [_p, _i64, _i64, _i64, ctypes.c_uint16, _p, _i64, _p]
         lib.oracle_quant_group128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_quant_block128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_block_gemm.argtypes = [_p, _i64, _p, _p, _i64, _p,
@@ -145,6 +146,17 @@ def quant_per_tensor(x_bits: np.ndarray):
     q = np.empty((m, k), dtype=np.uint8)
     s = np.zeros(1, dtype=np.float32)
     _load().oracle_quant_per_tensor(_ptr(x_bits), m, k, ld, _ptr(q), k, _ptr(s))
+    return q, s[0]
+
+
+def quant_apply(x_bits: np.ndarray, amax_bits: int):
+    """(codes, scale) of the apply-only step for a given amax word (the bf16
+    bit pattern of the amax; its sign bit is ignored)."""
+    m, k, ld = _rows(x_bits, 2)
+    q = np.empty((m, k), dtype=np.uint8)
+    s = np.zeros(1, dtype=np.float32)
+    _load().oracle_quant_apply(_ptr(x_bits), m, k, ld, ctypes.c_uint16(int(amax_bits) & 0xFFFF),
+                               _ptr(q), k, _ptr(s))
     return q, s[0]
 
 

@@ -238,6 +238,19 @@ void oracle_quant_per_tensor(const uint16_t* x, int64_t M, int64_t K, int64_t ld
             q[r * ldq + c] = quant_one(x[r * ldx + c], s);
 }
 
+/* The apply-only step of the per-tensor path ([P2] Description: a separate
+   pass quantises the input with the scale computed from the amax): amax is
+   given as the bf16 bit pattern of its magnitude. */
+void oracle_quant_apply(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                        uint16_t amax_bits, uint8_t* q, int64_t ldq, float* scale_out) {
+    float s = oracle_scale_from_amax(bf16_bits_to_f32((uint16_t)(amax_bits & 0x7FFF)));
+    *scale_out = s;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; r++)
+        for (int64_t c = 0; c < K; c++)
+            q[r * ldq + c] = quant_one(x[r * ldx + c], s);
+}
+
 /* Per-1x128-group quantisation along K ([P1] act_quant with block_size 128):
    for every row m and group g, amax over x[m, 128g : 128g+128], its own
    scale, and codes.  scales is [M, K/128] row-major. */
@@ -318,7 +331,7 @@ void oracle_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                        int64_t M, int64_t N, int64_t K, double* R, double* T) {
     double dec[256];
     decode_table(dec);
-    #pragma omp parallel for schedule(dynamic, 1)
+    #pragma omp parallel for collapse(2) schedule(static)
     for (int64_t m = 0; m < M; m++) {
         for (int64_t n = 0; n < N; n++) {
             double r, t;

@@ -402,3 +402,16 @@ def test_f64_to_bf16_matches_torch(oracle_mod):
 def test_tolerance_formula(oracle_mod):
     tol = oracle_mod.gemm_tolerance(np.array([1.0, 1.5, -3.0, 0.0]), np.zeros(4))
     np.testing.assert_array_equal(tol, [2 * 2.0 ** -7, 2 * 2.0 ** -7, 2 * 2.0 ** -6, 2 * 2.0 ** -133])
+
+
+def test_quant_apply_matches_per_tensor(oracle_mod):
+    x = inputs.activations_per_tensor(64)
+    bits = inputs.bf16_bits(x)
+    q1, s1 = oracle_mod.quant_per_tensor(bits)
+    word = int((bits & 0x7FFF).max())
+    q2, s2 = oracle_mod.quant_apply(bits, word)
+    assert s1 == s2
+    np.testing.assert_array_equal(q1, q2)
+    q3, s3 = oracle_mod.quant_apply(bits, 0)
+    assert s3 == 0
+    np.testing.assert_array_equal(q3, np.where(np.signbit(x.float().numpy()), 0x80, 0).astype(np.uint8))
