@@ -87,8 +87,9 @@ def activations_per_tensor(m: int, seed: int | None = None,
     x = g.standard_normal((m, k))
     rows = np.arange(0, m, 16)
     x[rows, :] *= g.uniform(1.0, 100.0, size=rows.size)[:, None]
-    grp = int(g.integers(0, k // 128))
-    x[m // 2, 128 * grp:128 * grp + 128] = 0.0
+    if k >= 128:
+        grp = int(g.integers(0, k // 128))
+        x[m // 2, 128 * grp:128 * grp + 128] = 0.0
     return to_bf16(x)
 
 
