@@ -15,6 +15,11 @@
 #include "gemm_kernels.cuh"
 #include "quant_kernels.cuh"
 
+// Split-K partial sums of fp8_block_gemm_noalloc live in this file-scope
+// device array instead of a caller-provided workspace.  Every device that
+// loads the library holds it until the process exits.
+static __device__ __align__(256) float g_noalloc_scratch[FP8Q_NOALLOC_MAX_SCRATCH_BYTES / sizeof(float)];
+
 namespace fp8q {
 namespace {
 
@@ -215,6 +220,34 @@ void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams&
                  cudaStream_t st) {
     using C = GemmCfg<BN, SWAP, STAGES>;
     block_gemm_kernel<BN, SWAP, STAGES><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+}
+
+// ------------------------------------------------------------------ no-alloc GEMM scratch
+constexpr size_t kNoAllocScratchBytes = FP8Q_NOALLOC_MAX_SCRATCH_BYTES;
+
+// Device address of g_noalloc_scratch on the current device.  In host code
+// the symbol's name is only a host-side stand-in, so the address is looked
+// up once per device (with that device current) and cached.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+int noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return FP8Q_ERR_NO_DEVICE;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, ::g_noalloc_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return FP8Q_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return FP8Q_OK;
 }
 
 }  // namespace
@@ -481,6 +514,22 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
         rc = launch_status();
     }
     return rc;
+}
+
+// ------------------------------------------------------------ GEMM, no allocation
+int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb,
+                           int64_t ldb, const float* sb, void* y, int64_t ldy, int64_t M, int64_t N,
+                           int64_t K, void* stream) {
+    // Shape/pointer errors are reported exactly as fp8_block_gemm reports them.
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
+    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    if (fp8_block_gemm_workspace_size(M, N, K) > kNoAllocScratchBytes) return FP8Q_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != FP8Q_OK) return rc;
+    return fp8_block_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, scratch, kNoAllocScratchBytes,
+                          stream);
 }
 
 // ------------------------------------------------------------ status

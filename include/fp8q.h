@@ -170,6 +170,43 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Block-scaled FP8 GEMM without any allocation                         */
+/* ------------------------------------------------------------------ */
+
+/* The pages have no counterpart to this call; it exists for callers that
+ * cannot allocate device memory: code running while a stream is being
+ * captured (where cudaMalloc is not allowed), host frameworks and plugin
+ * interfaces that hand a kernel only its input and output buffers, and
+ * latency-critical loops that cannot afford cudaMalloc/cudaFree (cudaFree
+ * synchronises the device).
+ *
+ * Same operation, arguments, layouts and errors as fp8_block_gemm, minus
+ * the workspace.  The split-K partial sums that fp8_block_gemm would put in
+ * the caller's workspace go to a fixed scratch array inside the library
+ * instead: FP8Q_NOALLOC_MAX_SCRATCH_BYTES (8 MiB) per device, reserved by
+ * every device that loads the library until the process exits.  Shapes
+ * whose launch needs more scratch than that (fp8_block_gemm_workspace_size
+ * (M,N,K) > FP8Q_NOALLOC_MAX_SCRATCH_BYTES) are rejected with
+ * FP8Q_ERR_WORKSPACE before anything is enqueued; use fp8_block_gemm for
+ * them.
+ *
+ * The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ * library routine.  The first call on each device looks up the scratch
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture begins.
+ *
+ * All calls on a device share the one scratch array, which keeps the last
+ * call's contents; each call overwrites every partial sum it reads, so no
+ * clearing is needed.  Two calls whose executions overlap on the GPU (e.g.
+ * on different streams without ordering) race on the scratch array and may
+ * produce wrong results: order them. */
+#define FP8Q_NOALLOC_MAX_SCRATCH_BYTES ((size_t)8 << 20)
+int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa,
+                           const uint8_t* qb, int64_t ldb, const float* sb,
+                           void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Device status                                                       */
 /* ------------------------------------------------------------------ */
 

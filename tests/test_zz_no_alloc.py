@@ -1,0 +1,69 @@
+"""fp8_block_gemm_noalloc: the block GEMM for callers that cannot allocate
+device memory (code running under stream capture, plugin hosts that hand over
+only input and output buffers, loops that cannot pay for cudaMalloc/cudaFree).
+Its split-K scratch is a fixed array inside the library instead of a caller
+workspace.
+
+Called through the C ABI (ctypes) and checked against the allocating entry
+point fp8_block_gemm on two calls in a row with different inputs -- the
+second call must not see the first call's leftovers in the shared scratch --
+within the GEMM tolerance the other tests use.  This file is collected last
+so a stop-at-first-failure run has already run every other test.
+"""
+import numpy as np
+import pytest
+import torch
+
+from fp8_dynamic_quantization_b200 import _abi, inputs
+import fp8_dynamic_quantization_b200 as fq
+
+pytestmark = pytest.mark.gpu
+
+FP8Q_OK, FP8Q_ERR_WORKSPACE = 0, 4
+
+
+def _noalloc(lib, qa, sa, qb, sb, y):
+    M, K = qa.shape
+    N = qb.shape[0]
+    return lib.fp8_block_gemm_noalloc(qa.data_ptr(), qa.stride(0), sa.data_ptr(), qb.data_ptr(),
+                                      qb.stride(0), sb.data_ptr(), y.data_ptr(), y.stride(0), M, N, K,
+                                      torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(a, gpu):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(gpu)
+
+
+@pytest.mark.parametrize("m,n,k", [(16, 2048, 7168), (64, 7168, 7168), (3, 200, 1024)])
+def test_noalloc_matches_allocating_gemm_twice(oracle_mod, cuda_lib, gpu, m, n, k):
+    lib = _abi.load()
+    need = lib.fp8_block_gemm_workspace_size(m, n, k)
+    assert 0 < need <= _abi.NOALLOC_MAX_SCRATCH_BYTES      # these shapes use split-K scratch
+    for call, seed in enumerate((101, 202)):
+        qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=seed + m + n)
+        tqa, tsa, tqb, tsb = (_dev(a, gpu) for a in (qa, sa, qb, sb))
+        ldy = (n + 7) // 8 * 8
+        y = torch.full((m, ldy), float("nan"), dtype=torch.bfloat16, device=gpu)[:, :n]
+        assert _noalloc(lib, tqa, tsa, tqb, tsb, y) == FP8Q_OK
+        y_ref = fq.block_gemm(tqa, tsa, tqb, tsb)
+        torch.cuda.synchronize()
+        Y = y.float().cpu().numpy().astype(np.float64)
+        Yr = y_ref.float().cpu().numpy().astype(np.float64)
+        _, T = oracle_mod.block_gemm(qa, sa, qb, sb)
+        tol = oracle_mod.gemm_tolerance(Yr, T)
+        assert np.all(np.abs(Y - Yr) <= tol), f"call {call}: noalloc result differs"
+    assert fq.device_status() == 0
+
+
+def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_lib, gpu):
+    lib = _abi.load()
+    m, n, k = 120, 2048, 7168
+    assert lib.fp8_block_gemm_workspace_size(m, n, k) > _abi.NOALLOC_MAX_SCRATCH_BYTES
+    qa = torch.zeros(m, k, dtype=torch.uint8, device=gpu)
+    sa = torch.ones(m, k // 128, dtype=torch.float32, device=gpu)
+    qb = torch.zeros(n, k, dtype=torch.uint8, device=gpu)
+    sb = torch.ones((n + 127) // 128, k // 128, dtype=torch.float32, device=gpu)
+    y = torch.full((m, n), 3.0, dtype=torch.bfloat16, device=gpu)
+    assert _noalloc(lib, qa, sa, qb, sb, y) == FP8Q_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert torch.all(y == 3.0)                 # nothing was enqueued
