@@ -304,18 +304,21 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
     uint32_t* ws = static_cast<uint32_t*>(workspace);
     const int64_t fused_grid = (nvec + int64_t(kQuantThreads) * kFusedU - 1) /
                                (int64_t(kQuantThreads) * kFusedU);
-    if (fused_grid <= std::min<int64_t>(d->fused_capacity, kMaxPartials)) {
-        int64_t spin = int64_t(1) << 24;
-        void* args[] = {(void*)&x, (void*)&nvec, (void*)&vpr, (void*)&ldx, (void*)&q,
-                        (void*)&ldq, (void*)&scale, (void*)&ws, (void*)&spin};
-        const void* fn = contig ? (const void*)per_tensor_fused_kernel<kFusedU, true>
-                                : (const void*)per_tensor_fused_kernel<kFusedU, false>;
+    // Single launch when every CTA fits on its own SM at once (all of them
+    // are resident together, so the grid barrier completes; it is bounded
+    // anyway and reports FP8Q_ERR_TIMEOUT instead of hanging).
+    if (fused_grid <= std::min<int64_t>(std::min(d->fused_capacity, d->sms), kMaxPartials)) {
+        const int64_t spin = int64_t(1) << 24;
+        const uint16_t* xs = static_cast<const uint16_t*>(x);
         if (log_enabled())
             std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: fused grid=%lld\n",
                          (long long)M, (long long)K, (long long)fused_grid);
-        const cudaError_t e = cudaLaunchCooperativeKernel(fn, dim3(unsigned(fused_grid)),
-                                                          dim3(kQuantThreads), args, 0, st);
-        if (e != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
+        if (contig)
+            per_tensor_fused_kernel<kFusedU, true><<<unsigned(fused_grid), kQuantThreads, 0, st>>>(
+                xs, nvec, vpr, ldx, q, ldq, scale, ws, spin);
+        else
+            per_tensor_fused_kernel<kFusedU, false><<<unsigned(fused_grid), kQuantThreads, 0, st>>>(
+                xs, nvec, vpr, ldx, q, ldq, scale, ws, spin);
         return launch_status(1);
     }
     const int grid = stream_grid(nvec, d->sms);
@@ -326,12 +329,12 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (contig) {
         amax_partial_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
-        apply_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials, grid,
-                                                                     q, ldq, scale);
+        apply_kernel<kStreamU, true, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials,
+                                                                            grid, q, ldq, scale);
     } else {
         amax_partial_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
-        apply_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials, grid,
-                                                                      q, ldq, scale);
+        apply_kernel<kStreamU, false, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials,
+                                                                             grid, q, ldq, scale);
     }
     return launch_status(2);
 }
@@ -385,11 +388,11 @@ int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
     const int grid = stream_grid(nvec, d->sms);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (ldx == K && ldq == K)
-        apply_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
-                                                                     q, ldq, scale);
+        apply_kernel<kStreamU, true, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+                                                                           q, ldq, scale);
     else
-        apply_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
-                                                                      q, ldq, scale);
+        apply_kernel<kStreamU, false, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+                                                                            q, ldq, scale);
     return launch_status();
 }
 
@@ -491,6 +494,7 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
     p.tiles_q = pl.tiles_q;
     p.splits = pl.splits;
     p.units = pl.units;
+    p.scale_vec4 = (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
                      (long long)M, (long long)N, (long long)K, pl.swap ? "swap" : "normal", pl.bn,

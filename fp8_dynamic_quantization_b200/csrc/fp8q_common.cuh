@@ -11,9 +11,26 @@
 //            every NaN sorts above +Inf, so the max is exact and NaN
 //            propagates -- independent of the reduction order.
 //   scale  = __fdiv_rn(amax, 448.f)           (one IEEE fp32 division)
-//   code   = cvt.rn.satfinite.e4m3x2.f32(__fdiv_rn(x, scale))
+//   code   = cvt.rn.satfinite.e4m3x2.f32(RN(x / scale))
 //            (round to nearest even, saturate to +-448, NaN -> 0x7F)
 //   scale == 0 (all-zero tensor or group): code = sign bit of x.
+//
+// RN(x / scale) without a division per element: with r = RN(1/scale)
+// (__frcp_rn, once per scale), q0 = RN(x*r), rem = x - q0*scale (one fma),
+// q = fma(rem, r, q0) -- Markstein's correction step (P. Markstein,
+// "Computation of elementary functions on the IBM RISC System/6000
+// processor", IBM J. Res. Dev. 34(1), 1990).  Here x is a bf16 value and
+// scale = RN(amax/448) with amax a bf16 value, so only 128 x 128 pairs of
+// significands can occur; the quotient is scale-invariant in the normal
+// range, and every pair was checked to give exactly RN(x/scale) (the test
+// suite also compares every (x, amax) pair of bf16 bit patterns with the
+// oracle's IEEE division on the GPU).  The scale must lie in [2^-90, 2^126]:
+// then any quotient that can give a nonzero code (>= 2^-10) has |x| >=
+// 2^-100, so the remainder is a normal number and exact, and smaller
+// quotients stay below 2^-10 (a signed-zero code) even where a subnormal x
+// makes the remainder inexact.  Other scales (tiny, infinite, NaN) and
+// inputs above the amax (possible only when the caller supplies the amax)
+// take __fdiv_rn instead.
 #pragma once
 
 #include <cstdint>
@@ -52,9 +69,29 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
-// Codes of one bf16 pair under scale s (s != 0).
-__device__ __forceinline__ uint32_t quant_pair(uint32_t w, float s) {
-    return cvt_e4m3x2(__fdiv_rn(bf16_lo(w), s), __fdiv_rn(bf16_hi(w), s));
+// A scale and what dividing by it needs.
+struct Scale {
+    float s;      // the scale
+    float r;      // RN(1/s)
+    int mode;     // 0: s == 0; 1: reciprocal-corrected division; 2: IEEE division
+};
+
+__device__ __forceinline__ Scale make_scale(float s) {
+    Scale d;
+    d.s = s;
+    d.r = __frcp_rn(s);
+    d.mode = (s == 0.0f) ? 0 : (s >= 0x1p-90f && s <= 0x1p126f) ? 1 : 2;
+    return d;
+}
+
+// RN(x / s) for finite |x| <= amax and 2^-90 <= s <= 2^126 (see above).
+// The remainder is formed negated, q0*s - x, so that x = -0 yields -0
+// ((-0) + (+0) would round to +0 in the other order); for every nonzero
+// quotient the result is the same, round-to-nearest being sign-symmetric.
+__device__ __forceinline__ float div_fast(float x, const Scale& d) {
+    const float q0 = __fmul_rn(x, d.r);
+    const float nrem = __fmaf_rn(q0, d.s, -x);
+    return __fmaf_rn(-nrem, d.r, q0);
 }
 
 // Signed-zero codes of one bf16 pair (the zero-scale convention).
@@ -62,16 +99,25 @@ __device__ __forceinline__ uint32_t zero_pair(uint32_t w) {
     return ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
 }
 
-// Codes of 8 bf16 values (one 16-byte vector) -> 8 bytes.
-__device__ __forceinline__ uint2 quant8(const uint4& v, float s) {
+// Codes of 8 bf16 values (one 16-byte vector) -> 8 bytes.  `exact` forces
+// the IEEE division (for values that may exceed the amax).
+__device__ __forceinline__ uint2 quant8(const uint4& v, const Scale& d, bool exact = false) {
     uint2 r;
-    if (s != 0.0f) {
-        r.x = quant_pair(v.x, s) | (quant_pair(v.y, s) << 16);
-        r.y = quant_pair(v.z, s) | (quant_pair(v.w, s) << 16);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c[4];
+    if (d.mode == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = zero_pair(w[i]);
+    } else if (d.mode == 1 && !exact) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(div_fast(bf16_lo(w[i]), d), div_fast(bf16_hi(w[i]), d));
     } else {
-        r.x = zero_pair(v.x) | (zero_pair(v.y) << 16);
-        r.y = zero_pair(v.z) | (zero_pair(v.w) << 16);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            c[i] = cvt_e4m3x2(__fdiv_rn(bf16_lo(w[i]), d.s), __fdiv_rn(bf16_hi(w[i]), d.s));
     }
+    r.x = c[0] | (c[1] << 16);
+    r.y = c[2] | (c[3] << 16);
     return r;
 }
 

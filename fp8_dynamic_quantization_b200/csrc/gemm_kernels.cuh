@@ -8,24 +8,30 @@
 //
 // The scales are arbitrary fp32 values, not powers of two, so the tensor
 // cores cannot apply them: each 128-wide K block is multiplied into a fresh
-// TMEM accumulator, and the promotion warps read that block's partial sum
-// (tcgen05.ld), multiply it by sa*sb in fp32 and add it to an fp32 running
-// sum held in registers.  Two TMEM buffers ping-pong so the MMA of block
-// kb+1 overlaps the promotion of block kb.
+// TMEM accumulator buffer, and the promotion warps read that block's partial
+// sum (tcgen05.ld), multiply it by sa*sb and add it to an fp32 running sum
+// held in registers (packed fma.rn.f32x2).  kNumBuf TMEM buffers rotate so
+// the MMAs of the next K blocks overlap the promotion of this one.
 //
 // Warp roles (one CTA per SM, persistent over work units):
-//   warp 0      TMA producer: P and Q tiles of one K block per pipeline stage
-//   warp 1      TMEM allocation; one thread issues tcgen05.mma (4 x K=32)
-//   warps 2..   promotion / epilogue, 128 threads per 128 accumulator columns
+//   warpgroup 0   warp 0: TMA producer (P and Q tiles of one K block per
+//                 pipeline stage); warp 1: TMEM allocation and the single
+//                 thread that issues tcgen05.mma; warps 2-3 idle.  With two
+//                 promotion warpgroups it hands registers to them
+//                 (setmaxnreg 40 / 232: 4*32*40 + 8*32*232 = 384*168).
+//   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row),
+//                 kCW accumulator columns; warpgroup w-1 owns columns
+//                 [(w-1)*kCW, w*kCW).
 //
 // Operand roles.  The MMA computes D[128 rows, BN cols] = P * Q^T with P and
-// Q K-major tiles in shared memory.
+// Q K-major tiles in shared memory (128-byte swizzle).
 //   normal  (SWAP = false): P = A rows (m), Q = B rows (n).  Row scale
-//           sa[m,kb]; column scale sb[n/128,kb] is uniform per 128 columns.
+//           sa[m,kb]; column scale sb[n/128,kb] is uniform per 128 columns
+//           (BN = 224 tiles split per column).
 //   swapped (SWAP = true) : P = B rows (n), Q = A rows (m), for skinny M --
 //           the weight fills the 128-row MMA dimension and the few tokens
-//           become the MMA's N.  Row scale sb[n/128,kb] is uniform per tile;
-//           column scales sa[m,kb] are staged in shared memory per unit.
+//           become the MMA's N.  The per-column scale sa[m,kb]*sb[tile,kb]
+//           is computed once per work unit into shared memory.
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
 #pragma once
@@ -44,22 +50,31 @@ struct GemmParams {
     int64_t ldy, ldw;
     int M, N, G;
     int tiles_p, tiles_q, splits, units;
+    int scale_vec4;      // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
 };
 
 template <int BN, bool SWAP, int STAGES>
 struct GemmCfg {
     static constexpr int kEpiWG = BN > 128 ? 2 : 1;            // promotion warpgroups
-    static constexpr int kCW = BN > 128 ? 128 : BN;            // columns per thread
-    static constexpr int kThreads = 64 + 128 * kEpiWG;
+    static constexpr int kCW = BN / kEpiWG;                    // columns per promotion thread
+    static constexpr int kThreads = 128 + 128 * kEpiWG;
     static constexpr int kPBytes = 128 * 128;                  // 128 rows x 128 K bytes
     static constexpr int kQBytes = BN * 128;
     static constexpr int kStageBytes = kPBytes + kQBytes;
-    static constexpr int kTmemCols = (2 * BN) < 32 ? 32 : 2 * BN;
-    static constexpr int kSlabFloats = SWAP ? (32768 / 4) : 0; // swapped-mode sa slab
+    static constexpr int kNumBuf = (512 / BN) < 8 ? (512 / BN) : 8;
+    static constexpr int kTmemCols = kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
+                                   : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
+    static constexpr int kSlabFloats = SWAP ? (32768 / 4) : 0; // swapped-mode scale slab
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
                                          + size_t(kSlabFloats) * 4 + 256;
-    static_assert(BN == 16 || BN == 32 || BN == 64 || BN == 128 || BN == 256, "BN");
+    static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
+    static_assert(kCW % 16 == 0, "columns per thread");
     static_assert(!SWAP || BN <= 128, "swapped tiles hold at most 128 tokens");
+    // normal mode: each promotion slice must lie inside one 128-column
+    // weight-scale block (its column scale is uniform)
+    static_assert(SWAP || kCW == 128, "normal-mode tiles are 128 or 256 wide");
+    static_assert(kStageBytes % 1024 == 0, "stage alignment");
+    static_assert(kSmemBytes <= 232448, "shared memory");
 };
 
 __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp, int& tq,
@@ -72,11 +87,47 @@ __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp,
     kb1 = int((int64_t(split + 1) * p.G) / p.splits);
 }
 
+// acc[j] += v[j] * s for j in [0, n), n even, in packed pairs.
+template <int N>
+__device__ __forceinline__ void fma_uniform(float* acc, const float* v, float s) {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) ptx::fma2(acc[j], acc[j + 1], v[j], v[j + 1], s, s);
+}
+
+// acc[j] += v[j] * sl[j] with per-column scales from shared memory.
+template <int N>
+__device__ __forceinline__ void fma_columns(float* acc, const float* v, const float* sl) {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) {
+        const float2 s = *reinterpret_cast<const float2*>(sl + j);
+        ptx::fma2(acc[j], acc[j + 1], v[j], v[j + 1], s.x, s.y);
+    }
+}
+
+// Scales of 4 consecutive K blocks [4*g4, 4*g4+4) of one scale row
+// (zeros past G or for an absent row).
+__device__ __forceinline__ float4 load_scale4(const float* row, int g4, int G, bool vec4, bool valid) {
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int k0 = 4 * g4;
+    if (!valid || k0 >= G) return r;
+    if (vec4) return __ldg(reinterpret_cast<const float4*>(row + k0));
+    r.x = __ldg(row + k0);
+    if (k0 + 1 < G) r.y = __ldg(row + k0 + 1);
+    if (k0 + 2 < G) r.z = __ldg(row + k0 + 2);
+    if (k0 + 3 < G) r.w = __ldg(row + k0 + 3);
+    return r;
+}
+
+__device__ __forceinline__ float pick4(const float4& v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
+}
+
 template <int BN, bool SWAP, int STAGES>
 __global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES>::kThreads, 1)
 block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmQ, const GemmParams p) {
     using C = GemmCfg<BN, SWAP, STAGES>;
+    constexpr int NB = C::kNumBuf;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -84,18 +135,18 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     float* slab = reinterpret_cast<float*>(smem + size_t(STAGES) * C::kStageBytes);
     uint64_t* bars = reinterpret_cast<uint64_t*>(
         smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4);
-    uint64_t* full = bars;                   // [STAGES] TMA landed
-    uint64_t* empty = bars + STAGES;         // [STAGES] MMA done reading
-    uint64_t* tfull = bars + 2 * STAGES;     // [2] block partial ready in TMEM
-    uint64_t* tempty = bars + 2 * STAGES + 2;// [2] promotion done reading TMEM
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 4);
+    uint64_t* full = bars;                        // [STAGES] TMA landed
+    uint64_t* empty = bars + STAGES;              // [STAGES] MMA done reading
+    uint64_t* tfull = bars + 2 * STAGES;          // [NB] block partial ready in TMEM
+    uint64_t* tempty = bars + 2 * STAGES + NB;    // [NB] promotion done reading TMEM
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2 * NB);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&full[s], 1); ptx::mbar_init(&empty[s], 1); }
-        for (int b = 0; b < 2; ++b) { ptx::mbar_init(&tfull[b], 1); ptx::mbar_init(&tempty[b], 4 * C::kEpiWG); }
+        for (int b = 0; b < NB; ++b) { ptx::mbar_init(&tfull[b], 1); ptx::mbar_init(&tempty[b], 4 * C::kEpiWG); }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
@@ -108,9 +159,10 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 
     auto fail = [&]() { *abort_flag = 1; record_error(6 /* FP8Q_ERR_TIMEOUT */); };
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
+    if (warp < 4) {
+        if (C::kEpiWG == 2) ptx::regs_dec<40>();
+        if (warp == 0 && lane == 0) {
+            // -------------------------------------------------------- producer
             uint32_t it = 0;
             for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
                 int tp, tq, kb0, kb1;
@@ -124,7 +176,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     ptx::tma_load_2d(dst, &tmP, &full[s], kb * 128, tp * 128);
                     ptx::tma_load_2d(dst + C::kPBytes, &tmQ, &full[s], kb * 128, tq * BN);
                 }
-                if (*abort_flag) break;
             }
             if (*abort_flag) {
                 // Let this thread's own copies land before the CTA exits.
@@ -132,11 +183,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 for (uint32_t j = first; j < it; ++j)
                     ptx::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 100000000LL);
             }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
-        if (lane == 0) {
+        } else if (warp == 1 && lane == 0) {
+            // -------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BN);
             uint32_t it = 0, c = 0;
             for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
@@ -145,7 +193,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 for (int kb = kb0; kb < kb1; ++kb, ++it, ++c) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    const uint32_t buf = c & 1, tph = (c >> 1) & 1;
+                    const uint32_t buf = c % NB, tph = (c / NB) & 1;
                     if (!ptx::mbar_wait(&tempty[buf], tph ^ 1)) { fail(); break; }
                     if (!ptx::mbar_wait(&full[s], ph)) { fail(); break; }
                     ptx::tc_fence_after();
@@ -159,91 +207,120 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     ptx::mma_commit(&empty[s]);
                     ptx::mma_commit(&tfull[buf]);
                 }
-                if (*abort_flag) break;
             }
             if (*abort_flag && c > 0)
-                ptx::mbar_wait(&tfull[(c - 1) & 1], ((c - 1) >> 1) & 1, 100000000LL);
+                ptx::mbar_wait(&tfull[(c - 1) % NB], ((c - 1) / NB) & 1, 100000000LL);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------ promotion
-        const int e = warp - 2;                   // 0 .. 4*kEpiWG-1
+        if (C::kEpiWG == 2) ptx::regs_inc<232>();
+        const int e = warp - 4;                   // 0 .. 4*kEpiWG-1
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
-        const int chalf = e >> 2;                 // which 128-column half (BN = 256)
+        const int chalf = e >> 2;                 // which kCW-column slice
         const int row = quarter * 32 + lane;      // TMEM lane = tile row
         const int nthreads = 128 * C::kEpiWG;
-        const int etid = threadIdx.x - 64;
+        const int etid = threadIdx.x - 128;
+        const bool vec4 = p.scale_vec4 != 0;
         uint32_t c = 0;
         float acc[C::kCW];
         for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
             int tp, tq, kb0, kb1;
             unit_coords(p, u, tp, tq, kb0, kb1);
             const int nkb = kb1 - kb0;
-            // Scale sources for this unit.
-            const int m_row = tp * 128 + row;                  // normal: token row
-            const int n_row = tp * 128 + row;                  // swapped: weight row
             const int q0 = tq * BN;
+            const int m_row = tp * 128 + row;                 // normal: token row
+            const int n_row = tp * 128 + row;                 // swapped: weight row
             if (SWAP) {
-                // slab[kbl * BN + j] = sa[q0 + j, kb0 + kbl]
+                // slab[kbl*BN + j] = sa[q0+j, kb0+kbl] * sb[tp, kb0+kbl]
                 ptx::named_bar_sync(1, nthreads);
                 for (int i = etid; i < nkb * BN; i += nthreads) {
                     const int kbl = i / BN, j = i - kbl * BN;
                     const int m = q0 + j;
-                    slab[i] = (m < p.M) ? __ldg(p.sa + int64_t(m) * p.G + kb0 + kbl) : 0.0f;
+                    const int kb = kb0 + kbl;
+                    slab[i] = (m < p.M) ? __ldg(p.sa + int64_t(m) * p.G + kb) *
+                                          __ldg(p.sb + int64_t(tp) * p.G + kb)
+                                        : 0.0f;
                 }
                 ptx::named_bar_sync(1, nthreads);
             }
 #pragma unroll
             for (int j = 0; j < C::kCW; ++j) acc[j] = 0.0f;
 
-            // Scale of K block kb for this thread (normal mode) / tile (swapped).
-            auto row_scale = [&](int kb) -> float {
-                if (SWAP) return __ldg(p.sb + int64_t(tp) * p.G + kb);
-                const int nb = (q0 + chalf * 128) >> 7;
-                const float sbv = (nb * 128 < p.N) ? __ldg(p.sb + int64_t(nb) * p.G + kb) : 0.0f;
-                const float sav = (m_row < p.M) ? __ldg(p.sa + int64_t(m_row) * p.G + kb) : 0.0f;
-                return sav * sbv;
-            };
-            float s_next = row_scale(kb0);
+            // Normal mode: row scale sa[m_row, kb] times the column block's
+            // sb[nb, kb], fetched four K blocks at a time, one group ahead.
+            const int nb = (q0 + chalf * C::kCW) >> 7;
+            const bool row_ok = !SWAP && m_row < p.M;
+            const bool col_ok = !SWAP && nb * 128 < p.N;
+            const float* sa_row = p.sa + int64_t(SWAP ? 0 : (row_ok ? m_row : 0)) * p.G;
+            const float* sb_row = p.sb + int64_t(col_ok ? nb : 0) * p.G;
+            float4 sa_cur, sb_cur, sa_nxt, sb_nxt;
+            if (!SWAP) {
+                sa_cur = load_scale4(sa_row, kb0 >> 2, p.G, vec4, row_ok);
+                sb_cur = load_scale4(sb_row, kb0 >> 2, p.G, vec4, col_ok);
+                sa_nxt = load_scale4(sa_row, (kb0 >> 2) + 1, p.G, vec4, row_ok);
+                sb_nxt = load_scale4(sb_row, (kb0 >> 2) + 1, p.G, vec4, col_ok);
+            }
             bool ok = true;
             for (int kb = kb0; kb < kb1; ++kb, ++c) {
-                const float s_cur = s_next;
-                if (kb + 1 < kb1) s_next = row_scale(kb + 1);
-                const uint32_t buf = c & 1, tph = (c >> 1) & 1;
+                float s = 0.0f;
+                if (!SWAP) {
+                    if ((kb & 3) == 0 && kb != kb0) {
+                        sa_cur = sa_nxt;
+                        sb_cur = sb_nxt;
+                        sa_nxt = load_scale4(sa_row, (kb >> 2) + 1, p.G, vec4, row_ok);
+                        sb_nxt = load_scale4(sb_row, (kb >> 2) + 1, p.G, vec4, col_ok);
+                    }
+                    s = pick4(sa_cur, kb & 3) * pick4(sb_cur, kb & 3);
+                }
+                const uint32_t buf = c % NB, tph = (c / NB) & 1;
                 if (!ptx::mbar_wait(&tfull[buf], tph)) { fail(); ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16)
-                                       + buf * BN + chalf * 128;
-                const float* sl = slab + (kb - kb0) * BN;
-                if (C::kCW >= 32) {
+                                       + buf * BN + chalf * C::kCW;
+                const float* sl = slab + (kb - kb0) * BN + chalf * C::kCW;
+                // Chunks of 64, then 32, then 16 columns; the TMEM buffer is
+                // released right after the last load has landed.
+                constexpr int n64 = C::kCW / 64;
+                constexpr int r32 = (C::kCW % 64) / 32;
+                constexpr int r16 = (C::kCW % 32) / 16;
+                constexpr int nchunks = n64 + r32 + r16;
+                float v[64];
+                int col = 0, chunk = 0;
 #pragma unroll
-                    for (int cc = 0; cc < C::kCW / 32; ++cc) {
-                        float v[32];
-                        ptx::tmem_ld32(taddr + cc * 32, v);
-                        ptx::tmem_wait_ld();
-                        if (cc == C::kCW / 32 - 1) {
-                            ptx::tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-                        }
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const float sj = SWAP ? s_cur * sl[cc * 32 + j] : s_cur;
-                            acc[cc * 32 + j] = fmaf(v[j], sj, acc[cc * 32 + j]);
-                        }
+                for (int i = 0; i < n64; ++i, ++chunk) {
+                    ptx::tmem_ld64(taddr + col, v);
+                    ptx::tmem_wait_ld();
+                    if (chunk == nchunks - 1) {
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
                     }
-                } else {
-                    float v[16];
-                    ptx::tmem_ld16(taddr, v);
+                    if (SWAP) fma_columns<64>(acc + col, v, sl + col);
+                    else fma_uniform<64>(acc + col, v, s);
+                    col += 64;
+                }
+                if (r32) {
+                    ptx::tmem_ld32(taddr + col, v);
+                    ptx::tmem_wait_ld();
+                    if (chunk == nchunks - 1) {
+                        ptx::tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                    }
+                    if (SWAP) fma_columns<32>(acc + col, v, sl + col);
+                    else fma_uniform<32>(acc + col, v, s);
+                    col += 32;
+                    ++chunk;
+                }
+                if (r16) {
+                    ptx::tmem_ld16(taddr + col, v);
                     ptx::tmem_wait_ld();
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float sj = SWAP ? s_cur * sl[j] : s_cur;
-                        acc[j] = fmaf(v[j], sj, acc[j]);
-                    }
+                    if (SWAP) fma_columns<16>(acc + col, v, sl + col);
+                    else fma_uniform<16>(acc + col, v, s);
                 }
             }
             if (!ok) break;
@@ -252,7 +329,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             if (p.splits == 1) {
                 if (!SWAP) {
                     const int m = m_row;
-                    const int n_first = q0 + chalf * 128;
+                    const int n_first = q0 + chalf * C::kCW;
                     if (m < p.M) {
                         uint16_t* yr = p.y + int64_t(m) * p.ldy;
 #pragma unroll
@@ -290,7 +367,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 float* wsp = p.ws + int64_t(split) * p.M * p.ldw;
                 if (!SWAP) {
                     const int m = m_row;
-                    const int n_first = q0 + chalf * 128;
+                    const int n_first = q0 + chalf * C::kCW;
                     if (m < p.M) {
                         float* wr = wsp + int64_t(m) * p.ldw;
 #pragma unroll

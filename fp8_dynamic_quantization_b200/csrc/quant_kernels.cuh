@@ -75,10 +75,10 @@ group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            const float s = scale_from_amax(amax_bits_to_f32(m));
+            const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
             if (g < groups) {
-                st_stream8(q + qo[u], quant8(v[u], s));
-                if (sub == 0) scales[g] = s;
+                st_stream8(q + qo[u], quant8(v[u], d));
+                if (sub == 0) scales[g] = d.s;
             }
         }
     }
@@ -112,17 +112,20 @@ amax_partial_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_pe
 // ---------------------------------------------------------------------------
 // Per-tensor apply: amax = max(partials[0:nparts]); scale; codes.
 // ---------------------------------------------------------------------------
-template <int U, bool CONTIG>
+// CHECK: the amax comes from the caller, so a vector may hold values above
+// it (or Inf); such vectors take the IEEE division.
+template <int U, bool CONTIG, bool CHECK>
 __global__ void __launch_bounds__(kQuantThreads)
 apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, int64_t ldx,
              const uint32_t* __restrict__ partials, int nparts,
              uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale_out) {
     __shared__ uint32_t red[kQuantThreads / 32];
     uint32_t m = 0;
-    for (int i = threadIdx.x; i < nparts; i += kQuantThreads) m = max(m, __ldcg(partials + i));
+    for (int i = threadIdx.x; i < nparts; i += kQuantThreads)
+        m = max(m, __ldcg(partials + i) & 0x7FFFu);
     m = block_max<kQuantThreads>(m, red);
-    const float s = scale_from_amax(amax_bits_to_f32(m));
-    if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = s;
+    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
+    if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = d.s;
 
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
     const int64_t span = U * stride;
@@ -142,7 +145,7 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
             const int64_t i = i0 + u * stride;
             if (i < nvec) {
                 const int64_t qo = CONTIG ? i * 8 : vec_offset<false>(i, vec_per_row, ldq);
-                st_stream8(q + qo, quant8(v[u], s));
+                st_stream8(q + qo, quant8(v[u], d, CHECK && absmax8(v[u]) > m));
             }
         }
     }
@@ -195,7 +198,7 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
             int64_t n = 0;
             while (vws[1] == gen0) {
                 if (++n > spin_limit) { ok = 0; record_error(6 /* FP8Q_ERR_TIMEOUT */); break; }
-                __nanosleep(64);
+                __nanosleep(32);
             }
         }
         __threadfence();
@@ -207,14 +210,14 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
     uint32_t mm = 0;
     for (int i = threadIdx.x; i < int(gridDim.x); i += kQuantThreads) mm = max(mm, __ldcg(ws + 2 + i));
     mm = block_max<kQuantThreads>(mm, red);
-    const float s = scale_from_amax(amax_bits_to_f32(mm));
-    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = s;
+    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(mm)));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = d.s;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int64_t i = first + u * stride;
         if (i < nvec) {
             const int64_t qo = CONTIG ? i * 8 : vec_offset<false>(i, vec_per_row, ldq);
-            st_stream8(q + qo, quant8(v[u], s));
+            st_stream8(q + qo, quant8(v[u], d));
         }
     }
 }
@@ -255,14 +258,14 @@ block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
         m = max(m, absmax8(v[u]));
     }
     m = block_max<kQuantThreads>(m, red);
-    const float s = scale_from_amax(amax_bits_to_f32(m));
-    if (threadIdx.x == 0) sb[nb * G + kb] = s;
+    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
+    if (threadIdx.x == 0) sb[nb * G + kb] = d.s;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const int j = threadIdx.x + u * kQuantThreads;
         const int64_t r = nb * 128 + (j >> 4);
         const int c = (j & 15) * 8;
-        if (r < N) st_stream8(q + r * ldq + kb * 128 + c, quant8(v[u], s));
+        if (r < N) st_stream8(q + r * ldq + kb * 128 + c, quant8(v[u], d));
     }
 }
 

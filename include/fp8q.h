@@ -94,9 +94,10 @@ size_t fp8_act_quant_per_tensor_workspace_size(int64_t M, int64_t K);
 /* x: bf16 [M,K], row stride ldx.  Writes codes q: uint8 [M,K], row stride
  * ldq, and *scale (one fp32 on the device) = fl32(amax / 448), with
  * amax = max |x| over the whole tensor (exact).  K must be a multiple of 8.
- * M == 0 or K == 0 writes scale 0 and nothing else.  Small tensors take a
- * single launch with a bounded grid barrier; larger ones take an amax pass
- * with an input-sized grid and then an apply pass. */
+ * M == 0 or K == 0 writes scale 0 and nothing else.  Small tensors (one
+ * CTA per SM suffices) take a single launch with a bounded grid barrier;
+ * larger ones take an amax pass with an input-sized grid and then an apply
+ * pass that re-reads x in reverse order (its tail is still in L2). */
 int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx,
                              uint8_t* q, int64_t ldq, float* scale,
                              void* workspace, size_t workspace_bytes,

@@ -211,3 +211,29 @@ def test_block128_weight(oracle_mod, gpu, n, k):
 
 def test_no_device_errors_recorded(gpu):
     assert fq.device_status(reset=False) == 0
+
+
+def test_every_x_and_amax_pair(oracle_mod, gpu):
+    """Every bf16 value x against every non-negative amax word (2^31 pairs):
+    the kernels' division by the scale must give the oracle's codes for all
+    of them (including x above the amax, Inf, NaN, zero and subnormal
+    scales)."""
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(512, 128)
+    x_dev = torch.from_numpy(bits.view(np.int16).copy()).view(torch.bfloat16).to(gpu)
+    words = torch.arange(0x8000, dtype=torch.int32, device=gpu)
+    chunk = 1024
+    for w0 in range(0, 0x8000, chunk):
+        got = torch.empty(chunk, 512, 128, dtype=torch.uint8, device=gpu)
+        scales = torch.empty(chunk, dtype=torch.float32, device=gpu)
+        for i in range(chunk):
+            q, s = fq.act_quant_apply(x_dev, words[w0 + i:w0 + i + 1])
+            got[i] = q.view(torch.uint8)
+            scales[i] = s[0]
+        got_np = got.cpu().numpy()
+        s_np = scales.cpu().numpy()
+        for i in range(chunk):
+            want, s_ref = oracle_mod.quant_apply(bits, w0 + i)
+            if not (np.array_equal(got_np[i], want) and
+                    s_np[i].view(np.uint32) == np.float32(s_ref).view(np.uint32)):
+                assert_scales_equal(s_np[i:i + 1], np.array([s_ref]))
+                assert_codes_equal(got_np[i], want)
