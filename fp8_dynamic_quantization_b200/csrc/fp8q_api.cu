@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include "fp8q_status.cuh"
@@ -52,11 +53,11 @@ constexpr int kStreamU = 4;         // vectors per thread per iteration elsewher
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
 
-template <int BN, bool SWAP, int STAGES>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false>
 cudaError_t set_gemm_smem() {
-    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES>,
+    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(GemmCfg<BN, SWAP, STAGES>::kSmemBytes));
+                                int(GemmCfg<BN, SWAP, STAGES, PAIR>::kSmemBytes));
 }
 
 // Device facts, queried once per device.  FP8Q_ERR_NO_DEVICE unless the
@@ -92,12 +93,15 @@ int device_info(DeviceInfo** out) {
             d.fused_capacity = std::min(per_sm, per_sm_nc) * d.sms;
             if (d.status == FP8Q_OK) {
                 cudaError_t e = cudaSuccess;
-                if (e == cudaSuccess) e = set_gemm_smem<16, true, 6>();
-                if (e == cudaSuccess) e = set_gemm_smem<32, true, 6>();
-                if (e == cudaSuccess) e = set_gemm_smem<64, true, 6>();
-                if (e == cudaSuccess) e = set_gemm_smem<128, true, 5>();
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 12>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 10>();
+                if (e == cudaSuccess) e = set_gemm_smem<64, true, 8>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, true, 6>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6>();
+                if (e == cudaSuccess) e = set_gemm_smem<192, false, 5>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true>();
                 if (e != cudaSuccess) { cudaGetLastError(); d.status = FP8Q_ERR_CUDA; }
             }
             d.ready = true;
@@ -138,45 +142,77 @@ int check_bf16_matrix(const void* x, int64_t rows, int64_t cols, int64_t ldx,
 }
 
 // ------------------------------------------------------------------ GEMM plan
-enum Mode { kNormal = 0, kSwap = 1 };
+enum Mode { kNormal = 0, kSwap = 1, kPair = 2 };
 struct TableRow { int64_t m_lo, m_hi, n_lo, n_hi; int mode, bn, splits; };
 const TableRow kGemmTable[] = {
 #include "launch_table.inc"
 };
 
 struct GemmPlan {
-    bool swap;
+    bool swap, pair;
     int bn, stages, splits, tiles_p, tiles_q, units, grid;
     int64_t ldw;
     size_t ws_bytes;
 };
+
+// Tuning override of the table (FP8Q_GEMM_TILE="normal:128", "swap:64:4",
+// ...: mode, tile width, optional split-K count).  For measuring launch
+// choices only; every choice computes the same sums.
+bool tile_override(TableRow* out) {
+    static TableRow row;
+    static const bool has = [] {
+        const char* v = std::getenv("FP8Q_GEMM_TILE");
+        if (!v || !v[0]) return false;
+        char mode[16] = {0};
+        int bn = 0, splits = 0;
+        if (std::sscanf(v, "%15[a-z]:%d:%d", mode, &bn, &splits) < 2) return false;
+        const bool swap = std::strcmp(mode, "swap") == 0;
+        const bool pair = std::strcmp(mode, "pair") == 0;
+        if (!swap && !pair && std::strcmp(mode, "normal") != 0) return false;
+        if (swap ? !(bn == 16 || bn == 32 || bn == 64 || bn == 128)
+                 : pair ? !(bn == 256 || bn == 128) : !(bn == 128 || bn == 192 || bn == 256))
+            return false;
+        row = TableRow{1, int64_t(1) << 30, 1, int64_t(1) << 30, swap ? kSwap : pair ? kPair : kNormal,
+                       bn, pair ? 1 : splits};
+        return true;
+    }();
+    if (has) *out = row;
+    return has;
+}
 
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
     GemmPlan pl{};
     const TableRow* row = &kGemmTable[0];
     for (const TableRow& r : kGemmTable)
         if (M >= r.m_lo && M <= r.m_hi && N >= r.n_lo && N <= r.n_hi) { row = &r; break; }
+    TableRow forced;
+    if (tile_override(&forced)) row = &forced;
     pl.swap = row->mode == kSwap;
+    pl.pair = row->mode == kPair;
     pl.bn = row->bn;
-    pl.stages = pl.swap ? (pl.bn == 128 ? 5 : 6) : (pl.bn == 256 ? 4 : 6);
+    pl.stages = pl.swap ? (pl.bn == 16 ? 12 : pl.bn == 32 ? 10 : pl.bn == 64 ? 8 : 6)
+                        : pl.pair ? (pl.bn == 256 ? 6 : 8) : (pl.bn == 192 ? 5 : pl.bn == 256 ? 4 : 6);
     const int G = int(K / 128);
     const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
-    pl.tiles_p = int((rows_p + 127) / 128);
+    const int tile_rows = pl.pair ? 256 : 128;
+    pl.tiles_p = int((rows_p + tile_rows - 1) / tile_rows);
     pl.tiles_q = int((rows_q + pl.bn - 1) / pl.bn);
     const int64_t tiles = int64_t(pl.tiles_p) * pl.tiles_q;
     int splits = row->splits;
+    if (pl.pair) splits = 1;
     if (splits <= 0) {
         splits = 1;
         if (tiles < sms) splits = int(std::max<int64_t>(1, sms / tiles));
         splits = std::min(splits, std::max(1, G / 2));   // at least 2 K blocks per split
     }
     splits = std::max(1, std::min(splits, G));
-    if (pl.swap) {   // the swapped kernel stages ceil(G/splits) x bn scales in shared memory
-        while (((G + splits - 1) / splits) * pl.bn > 8192) ++splits;
+    if (pl.swap) {   // the swapped kernel stages at most 64 K blocks of scales per unit
+        while ((G + splits - 1) / splits > 64) ++splits;
     }
     pl.splits = splits;
     pl.units = int(tiles * splits);
-    pl.grid = std::max(1, std::min(pl.units, sms));
+    pl.grid = pl.pair ? 2 * std::max(1, std::min(pl.units, sms / 2))
+                      : std::max(1, std::min(pl.units, sms));
     pl.ldw = (N + 7) / 8 * 8;
     pl.ws_bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(pl.ldw) * sizeof(float) : 0;
     return pl;
@@ -215,11 +251,27 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWAP, int STAGES>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& p, int grid,
                  cudaStream_t st) {
-    using C = GemmCfg<BN, SWAP, STAGES>;
-    block_gemm_kernel<BN, SWAP, STAGES><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR>;
+    if (!PAIR) {
+        block_gemm_kernel<BN, SWAP, STAGES, PAIR><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+        return;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(unsigned(grid));
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR>, tp, tq, p);
 }
 
 // ------------------------------------------------------------------ no-alloc GEMM scratch
@@ -408,16 +460,17 @@ int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uin
     if ((rc = device_info(&d)) != FP8Q_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t G = K / 128, groups = M * G;
-    const int64_t need = (groups * 16 + int64_t(kQuantThreads) * kStreamU - 1) /
-                         (int64_t(kQuantThreads) * kStreamU);
+    constexpr int kGroupU = 2;        // groups per thread per iteration (8 threads a group)
+    const int64_t need = (groups * 8 + int64_t(kQuantThreads) * kGroupU - 1) /
+                         (int64_t(kQuantThreads) * kGroupU);
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(d->sms) * kBlocksPerSm)));
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] group128 M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (ldx == K && ldq == K)
-        group128_quant_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        group128_quant_kernel<kGroupU, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
     else
-        group128_quant_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        group128_quant_kernel<kGroupU, false><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
     return launch_status();
 }
 
@@ -478,7 +531,8 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
     const uint8_t* Q = pl.swap ? qa : qb;
     const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
     const int64_t ld_p = pl.swap ? ldb : lda, ld_q = pl.swap ? lda : ldb;
-    if (!make_tmap(&tp, P, rows_p, K, ld_p, 128) || !make_tmap(&tq, Q, rows_q, K, ld_q, pl.bn))
+    if (!make_tmap(&tp, P, rows_p, K, ld_p, 128) ||
+        !make_tmap(&tq, Q, rows_q, K, ld_q, pl.pair ? pl.bn / 2 : pl.bn))
         return FP8Q_ERR_CUDA;
     GemmParams p;
     p.sa = sa;
@@ -497,17 +551,22 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
     p.scale_vec4 = (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
-                     (long long)M, (long long)N, (long long)K, pl.swap ? "swap" : "normal", pl.bn,
+                     (long long)M, (long long)N, (long long)K,
+                     pl.swap ? "swap" : pl.pair ? "pair" : "normal", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
     if (pl.swap) {
         switch (pl.bn) {
-            case 16: launch_gemm<16, true, 6>(tp, tq, p, pl.grid, st); break;
-            case 32: launch_gemm<32, true, 6>(tp, tq, p, pl.grid, st); break;
-            case 64: launch_gemm<64, true, 6>(tp, tq, p, pl.grid, st); break;
-            default: launch_gemm<128, true, 5>(tp, tq, p, pl.grid, st); break;
+            case 16: launch_gemm<16, true, 12>(tp, tq, p, pl.grid, st); break;
+            case 32: launch_gemm<32, true, 10>(tp, tq, p, pl.grid, st); break;
+            case 64: launch_gemm<64, true, 8>(tp, tq, p, pl.grid, st); break;
+            default: launch_gemm<128, true, 6>(tp, tq, p, pl.grid, st); break;
         }
+    } else if (pl.pair) {
+        if (pl.bn == 256) launch_gemm<256, false, 6, true>(tp, tq, p, pl.grid, st);
+        else launch_gemm<128, false, 8, true>(tp, tq, p, pl.grid, st);
     } else {
-        if (pl.bn == 256) launch_gemm<256, false, 4>(tp, tq, p, pl.grid, st);
+        if (pl.bn == 192) launch_gemm<192, false, 5>(tp, tq, p, pl.grid, st);
+        else if (pl.bn == 256) launch_gemm<256, false, 4>(tp, tq, p, pl.grid, st);
         else launch_gemm<128, false, 6>(tp, tq, p, pl.grid, st);
     }
     if ((rc = launch_status()) != FP8Q_OK) return rc;

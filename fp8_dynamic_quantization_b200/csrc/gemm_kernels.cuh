@@ -10,24 +10,26 @@
 // cores cannot apply them: each 128-wide K block is multiplied into a fresh
 // TMEM accumulator buffer, and the promotion warps read that block's partial
 // sum (tcgen05.ld), multiply it by sa*sb and add it to an fp32 running sum
-// held in registers (packed fma.rn.f32x2).  kNumBuf TMEM buffers rotate so
+// held in registers as packed pairs (fma.rn.f32x2 in place).  kNumBuf TMEM buffers rotate so
 // the MMAs of the next K blocks overlap the promotion of this one.
 //
 // Warp roles (one CTA per SM, persistent over work units):
 //   warpgroup 0   warp 0: TMA producer (P and Q tiles of one K block per
 //                 pipeline stage); warp 1: TMEM allocation and the single
-//                 thread that issues tcgen05.mma; warps 2-3 idle.  With two
-//                 promotion warpgroups it hands registers to them
-//                 (setmaxnreg 40 / 232: 4*32*40 + 8*32*232 = 384*168).
-//   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row),
-//                 kCW accumulator columns; warpgroup w-1 owns columns
-//                 [(w-1)*kCW, w*kCW).
+//                 thread that issues tcgen05.mma; warps 2-3 idle.  With
+//                 several promotion warpgroups it hands registers to them
+//                 (setmaxnreg 48/224 or 56/216 for two, 32/160 for three).
+//   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row)
+//                 and a slice of kCW <= 64 accumulator columns; warpgroup
+//                 w-1 owns columns [(w-1)*kCW, w*kCW).  Each K block costs a
+//                 thread one tcgen05.ld and one wait before it releases the
+//                 TMEM buffer, which keeps the MMA <-> promotion hand-off
+//                 short; more warpgroups hide the load latency.
 //
 // Operand roles.  The MMA computes D[128 rows, BN cols] = P * Q^T with P and
 // Q K-major tiles in shared memory (128-byte swizzle).
 //   normal  (SWAP = false): P = A rows (m), Q = B rows (n).  Row scale
-//           sa[m,kb]; column scale sb[n/128,kb] is uniform per 128 columns
-//           (BN = 224 tiles split per column).
+//           sa[m,kb]; column scale sb[n/128,kb] is uniform per 128 columns.
 //   swapped (SWAP = true) : P = B rows (n), Q = A rows (m), for skinny M --
 //           the weight fills the 128-row MMA dimension and the few tokens
 //           become the MMA's N.  The per-column scale sa[m,kb]*sb[tile,kb]
@@ -53,28 +55,44 @@ struct GemmParams {
     int scale_vec4;      // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
 };
 
-template <int BN, bool SWAP, int STAGES>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false>
 struct GemmCfg {
-    static constexpr int kEpiWG = BN > 128 ? 2 : 1;            // promotion warpgroups
-    static constexpr int kCW = BN / kEpiWG;                    // columns per promotion thread
+    // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
+    // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
+    // and its TMEM receives its 128 rows x BN columns of every product.
+    static constexpr int kCW = BN == 256 ? 128 : (BN < 64 ? BN : 64);  // columns per promotion thread
+    static constexpr int kEpiWG = BN / kCW;                    // promotion warpgroups (1..3)
     static constexpr int kThreads = 128 + 128 * kEpiWG;
+    // Register split (setmaxnreg) between warpgroup 0 and the promotion
+    // warpgroups; it must add up to at most threads x launch registers.
+    static constexpr int kRegWG0 = kEpiWG == 2 ? (kCW == 128 ? 48 : 56) : 32;
+    static constexpr int kRegEpi = kEpiWG == 2 ? (kCW == 128 ? 224 : 216) : 160;
+    static constexpr int kLaunchRegs = ((65536 / kThreads) / 8) * 8 > 255 ? 255 : ((65536 / kThreads) / 8) * 8;
+    static_assert(kEpiWG == 1 || 128 * kRegWG0 + 128 * kEpiWG * kRegEpi <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
+    static_assert(kEpiWG <= 3, "at most three promotion warpgroups");
+    static constexpr int kTileRows = PAIR ? 256 : 128;         // rows of P per work unit
     static constexpr int kPBytes = 128 * 128;                  // 128 rows x 128 K bytes
-    static constexpr int kQBytes = BN * 128;
+    static constexpr int kQRows = PAIR ? BN / 2 : BN;         // B (or A) rows this CTA loads
+    static constexpr int kQBytes = kQRows * 128;
     static constexpr int kStageBytes = kPBytes + kQBytes;
     static constexpr int kNumBuf = (512 / BN) < 8 ? (512 / BN) : 8;
     static constexpr int kTmemCols = kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
-    static constexpr int kSlabFloats = SWAP ? (32768 / 4) : 0; // swapped-mode scale slab
+    static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
+    static constexpr int kSlabFloats = SWAP ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
-                                         + size_t(kSlabFloats) * 4 + 256;
+                                         + size_t(kSlabFloats) * 4 + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(kCW % 16 == 0, "columns per thread");
     static_assert(!SWAP || BN <= 128, "swapped tiles hold at most 128 tokens");
-    // normal mode: each promotion slice must lie inside one 128-column
-    // weight-scale block (its column scale is uniform)
-    static_assert(SWAP || kCW == 128, "normal-mode tiles are 128 or 256 wide");
+    // normal mode: each 64-column promotion slice starts at a multiple of 64,
+    // so it lies inside one 128-column weight-scale block (uniform scale)
+    static_assert(SWAP || kCW == 64 || kCW == 128, "normal-mode slices are 64 or 128 columns");
+    static_assert(!PAIR || (!SWAP && (BN == 256 || BN == 128)), "CTA pairs compute 256 x 256 or 256 x 128 tiles");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kSmemBytes <= 232448, "shared memory");
+    static_assert((2 * STAGES + 2 * kNumBuf) * 8 + 8 <= 512, "barrier area");
 };
 
 __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp, int& tq,
@@ -87,21 +105,22 @@ __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp,
     kb1 = int((int64_t(split + 1) * p.G) / p.splits);
 }
 
-// acc[j] += v[j] * s for j in [0, n), n even, in packed pairs.
+// Accumulators are kept as packed fp32 pairs: acc2[i] holds columns 2i and
+// 2i+1, so the packed fma.rn.f32x2 works on them in place.
+
+// acc2[j/2] += (v[j], v[j+1]) * (s, s) for j in [0, N).
 template <int N>
-__device__ __forceinline__ void fma_uniform(float* acc, const float* v, float s) {
+__device__ __forceinline__ void fma_uniform(uint64_t* acc2, const float* v, uint64_t s2) {
 #pragma unroll
-    for (int j = 0; j < N; j += 2) ptx::fma2(acc[j], acc[j + 1], v[j], v[j + 1], s, s);
+    for (int j = 0; j < N; j += 2) ptx::fma2p(acc2[j / 2], v[j], v[j + 1], s2);
 }
 
-// acc[j] += v[j] * sl[j] with per-column scales from shared memory.
+// acc2[j/2] += (v[j], v[j+1]) * (sl[j], sl[j+1]), scales from shared memory.
 template <int N>
-__device__ __forceinline__ void fma_columns(float* acc, const float* v, const float* sl) {
+__device__ __forceinline__ void fma_columns(uint64_t* acc2, const float* v, const float* sl) {
 #pragma unroll
-    for (int j = 0; j < N; j += 2) {
-        const float2 s = *reinterpret_cast<const float2*>(sl + j);
-        ptx::fma2(acc[j], acc[j + 1], v[j], v[j + 1], s.x, s.y);
-    }
+    for (int j = 0; j < N; j += 2)
+        ptx::fma2p(acc2[j / 2], v[j], v[j + 1], *reinterpret_cast<const uint64_t*>(sl + j));
 }
 
 // Scales of 4 consecutive K blocks [4*g4, 4*g4+4) of one scale row
@@ -122,11 +141,11 @@ __device__ __forceinline__ float pick4(const float4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int BN, bool SWAP, int STAGES>
-__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES>::kThreads, 1)
+template <int BN, bool SWAP, int STAGES, bool PAIR = false>
+__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR>::kThreads, 1)
 block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmQ, const GemmParams p) {
-    using C = GemmCfg<BN, SWAP, STAGES>;
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR>;
     constexpr int NB = C::kNumBuf;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -143,69 +162,106 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    // CTA pair: rank 0 (the leader) issues the MMAs; both load, both promote.
+    const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int unit0 = PAIR ? int(ptx::cluster_id_x()) : int(blockIdx.x);
+    const int unit_step = PAIR ? int(ptx::num_clusters_x()) : int(gridDim.x);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&full[s], 1); ptx::mbar_init(&empty[s], 1); }
-        for (int b = 0; b < NB; ++b) { ptx::mbar_init(&tfull[b], 1); ptx::mbar_init(&tempty[b], 4 * C::kEpiWG); }
+        for (int b = 0; b < NB; ++b) {
+            ptx::mbar_init(&tfull[b], 1);
+            ptx::mbar_init(&tempty[b], (PAIR ? 2 : 1) * 4 * C::kEpiWG);
+        }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmP); ptx::prefetch_tmap(&tmQ); }
-    if (warp == 1) { ptx::tmem_alloc(tmem_base_smem, C::kTmemCols); ptx::tmem_relinquish(); }
+    if (warp == 1) {
+        if (PAIR) { ptx::tmem_alloc_pair(tmem_base_smem, C::kTmemCols); ptx::tmem_relinquish_pair(); }
+        else { ptx::tmem_alloc(tmem_base_smem, C::kTmemCols); ptx::tmem_relinquish(); }
+    }
     ptx::tc_fence_before();
-    __syncthreads();
+    if (PAIR) ptx::cluster_sync();      // the peer may signal the leader's barriers from here on
+    else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
 
     auto fail = [&]() { *abort_flag = 1; record_error(6 /* FP8Q_ERR_TIMEOUT */); };
 
     if (warp < 4) {
-        if (C::kEpiWG == 2) ptx::regs_dec<40>();
+        if (C::kEpiWG > 1) ptx::regs_dec<C::kRegWG0>();
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- producer
             uint32_t it = 0;
-            for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
+            for (int u = unit0; u < p.units && !*abort_flag; u += unit_step) {
                 int tp, tq, kb0, kb1;
                 unit_coords(p, u, tp, tq, kb0, kb1);
+                const int prow = tp * C::kTileRows + int(rank) * 128;
+                const int qrow = tq * BN + int(rank) * C::kQRows;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     if (!ptx::mbar_wait(&empty[s], ph ^ 1)) { fail(); break; }
                     uint8_t* dst = tiles + size_t(s) * C::kStageBytes;
-                    ptx::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                    ptx::tma_load_2d(dst, &tmP, &full[s], kb * 128, tp * 128);
-                    ptx::tma_load_2d(dst + C::kPBytes, &tmQ, &full[s], kb * 128, tq * BN);
+                    if (PAIR) {
+                        // both CTAs' copies complete on the leader's barrier
+                        const uint32_t bar0 = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
+                        if (leader) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
+                        ptx::tma_load_2d_pair(dst, &tmP, bar0, kb * 128, prow);
+                        ptx::tma_load_2d_pair(dst + C::kPBytes, &tmQ, bar0, kb * 128, qrow);
+                    } else {
+                        ptx::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                        ptx::tma_load_2d(dst, &tmP, &full[s], kb * 128, prow);
+                        ptx::tma_load_2d(dst + C::kPBytes, &tmQ, &full[s], kb * 128, qrow);
+                    }
                 }
             }
-            if (*abort_flag) {
+            if (*abort_flag && leader) {
                 // Let this thread's own copies land before the CTA exits.
                 const uint32_t first = it > STAGES ? it - STAGES : 0;
                 for (uint32_t j = first; j < it; ++j)
                     ptx::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 100000000LL);
             }
-        } else if (warp == 1 && lane == 0) {
+        } else if (warp == 1 && lane == 0 && leader) {
             // -------------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BN);
+            constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BN, C::kTileRows);
             uint32_t it = 0, c = 0;
-            for (int u = blockIdx.x; u < p.units && !*abort_flag; u += gridDim.x) {
+            for (int u = unit0; u < p.units && !*abort_flag; u += unit_step) {
                 int tp, tq, kb0, kb1;
                 unit_coords(p, u, tp, tq, kb0, kb1);
                 for (int kb = kb0; kb < kb1; ++kb, ++it, ++c) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     const uint32_t buf = c % NB, tph = (c / NB) & 1;
-                    if (!ptx::mbar_wait(&tempty[buf], tph ^ 1)) { fail(); break; }
+                    const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1)
+                                            : ptx::mbar_wait(&tempty[buf], tph ^ 1);
+                    if (!freed) { fail(); break; }
                     if (!ptx::mbar_wait(&full[s], ph)) { fail(); break; }
                     ptx::tc_fence_after();
                     const uint32_t pa = ptx::smem_u32(tiles + size_t(s) * C::kStageBytes);
                     const uint32_t qa = pa + C::kPBytes;
                     const uint32_t d = tmem_base + buf * BN;
+                    if (PAIR) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        ptx::mma_f8(d, ptx::sw128_kmajor_desc(pa + 32 * k),
-                                    ptx::sw128_kmajor_desc(qa + 32 * k), idesc, k > 0);
-                    ptx::mma_commit(&empty[s]);
-                    ptx::mma_commit(&tfull[buf]);
+                        for (int k = 0; k < 4; ++k)
+                            ptx::mma_f8_pair(d, ptx::sw128_kmajor_desc(pa + 32 * k),
+                                             ptx::sw128_kmajor_desc(qa + 32 * k), idesc, k > 0);
+                        // stage free and partial ready, in both CTAs
+                        const uint32_t e0 = ptx::smem_u32(&empty[s]), f0 = ptx::smem_u32(&tfull[buf]);
+                        ptx::mma_commit_pair(e0);
+                        ptx::mma_commit_pair(ptx::mapa_shared(e0, 1));
+                        ptx::mma_commit_pair(f0);
+                        ptx::mma_commit_pair(ptx::mapa_shared(f0, 1));
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            ptx::mma_f8(d, ptx::sw128_kmajor_desc(pa + 32 * k),
+                                        ptx::sw128_kmajor_desc(qa + 32 * k), idesc, k > 0);
+                        ptx::mma_commit(&empty[s]);
+                        ptx::mma_commit(&tfull[buf]);
+                    }
                 }
             }
             if (*abort_flag && c > 0)
@@ -214,7 +270,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         __syncwarp();
     } else {
         // ------------------------------------------------------------ promotion
-        if (C::kEpiWG == 2) ptx::regs_inc<232>();
+        if (C::kEpiWG > 1) ptx::regs_inc<C::kRegEpi>();
         const int e = warp - 4;                   // 0 .. 4*kEpiWG-1
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int chalf = e >> 2;                 // which kCW-column slice
@@ -223,14 +279,16 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         const int etid = threadIdx.x - 128;
         const bool vec4 = p.scale_vec4 != 0;
         uint32_t c = 0;
-        float acc[C::kCW];
-        for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
+        uint64_t acc2[C::kCW / 2];
+        // the leader's tempty barriers, as cluster addresses (pair mode)
+        const uint32_t tempty0 = PAIR ? ptx::mapa_shared(ptx::smem_u32(tempty), 0) : 0u;
+        for (int u = unit0; u < p.units; u += unit_step) {
             int tp, tq, kb0, kb1;
             unit_coords(p, u, tp, tq, kb0, kb1);
             const int nkb = kb1 - kb0;
             const int q0 = tq * BN;
-            const int m_row = tp * 128 + row;                 // normal: token row
-            const int n_row = tp * 128 + row;                 // swapped: weight row
+            const int m_row = tp * C::kTileRows + int(rank) * 128 + row;   // normal: token row
+            const int n_row = tp * 128 + row;                              // swapped: weight row
             if (SWAP) {
                 // slab[kbl*BN + j] = sa[q0+j, kb0+kbl] * sb[tp, kb0+kbl]
                 ptx::named_bar_sync(1, nthreads);
@@ -245,7 +303,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 ptx::named_bar_sync(1, nthreads);
             }
 #pragma unroll
-            for (int j = 0; j < C::kCW; ++j) acc[j] = 0.0f;
+            for (int j = 0; j < C::kCW / 2; ++j) acc2[j] = 0ull;
 
             // Normal mode: row scale sa[m_row, kb] times the column block's
             // sb[nb, kb], fetched four K blocks at a time, one group ahead.
@@ -273,59 +331,43 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     }
                     s = pick4(sa_cur, kb & 3) * pick4(sb_cur, kb & 3);
                 }
+                const uint64_t s2 = ptx::pack_f32x2(s, s);
                 const uint32_t buf = c % NB, tph = (c / NB) & 1;
                 if (!ptx::mbar_wait(&tfull[buf], tph)) { fail(); ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16)
                                        + buf * BN + chalf * C::kCW;
                 const float* sl = slab + (kb - kb0) * BN + chalf * C::kCW;
-                // Chunks of 64, then 32, then 16 columns; the TMEM buffer is
-                // released right after the last load has landed.
-                constexpr int n64 = C::kCW / 64;
-                constexpr int r32 = (C::kCW % 64) / 32;
-                constexpr int r16 = (C::kCW % 32) / 16;
-                constexpr int nchunks = n64 + r32 + r16;
-                float v[64];
-                int col = 0, chunk = 0;
+                // Loads of this thread's kCW columns in chunks of at most 64;
+                // the TMEM buffer is released as soon as the last chunk has
+                // landed, then that chunk's FMAs run.
+                constexpr int kChunk = C::kCW >= 64 ? 64 : C::kCW;
+                constexpr int kChunks = C::kCW / kChunk;
+                float v[kChunk];
 #pragma unroll
-                for (int i = 0; i < n64; ++i, ++chunk) {
-                    ptx::tmem_ld64(taddr + col, v);
+                for (int ch = 0; ch < kChunks; ++ch) {
+                    if constexpr (kChunk == 64) ptx::tmem_ld64(taddr + ch * 64, v);
+                    else if constexpr (kChunk == 32) ptx::tmem_ld32(taddr, v);
+                    else ptx::tmem_ld16(taddr, v);
                     ptx::tmem_wait_ld();
-                    if (chunk == nchunks - 1) {
+                    if (ch == kChunks - 1) {
                         ptx::tc_fence_before();
                         __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
+                        if (lane == 0) {
+                            if (PAIR) ptx::mbar_arrive_cluster(tempty0 + buf * 8);
+                            else ptx::mbar_arrive(&tempty[buf]);
+                        }
                     }
-                    if (SWAP) fma_columns<64>(acc + col, v, sl + col);
-                    else fma_uniform<64>(acc + col, v, s);
-                    col += 64;
-                }
-                if (r32) {
-                    ptx::tmem_ld32(taddr + col, v);
-                    ptx::tmem_wait_ld();
-                    if (chunk == nchunks - 1) {
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-                    }
-                    if (SWAP) fma_columns<32>(acc + col, v, sl + col);
-                    else fma_uniform<32>(acc + col, v, s);
-                    col += 32;
-                    ++chunk;
-                }
-                if (r16) {
-                    ptx::tmem_ld16(taddr + col, v);
-                    ptx::tmem_wait_ld();
-                    ptx::tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&tempty[buf]);
-                    if (SWAP) fma_columns<16>(acc + col, v, sl + col);
-                    else fma_uniform<16>(acc + col, v, s);
+                    if (SWAP) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
+                    else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
                 }
             }
             if (!ok) break;
 
             // ---------------------------------------------------- epilogue
+            float acc[C::kCW];
+#pragma unroll
+            for (int j = 0; j < C::kCW / 2; ++j) ptx::unpack_f32x2(acc2[j], acc[2 * j], acc[2 * j + 1]);
             if (p.splits == 1) {
                 if (!SWAP) {
                     const int m = m_row;
@@ -355,7 +397,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     if (n < p.N) {
 #pragma unroll
                         for (int j = 0; j < C::kCW; ++j) {
-                            const int m = q0 + j;
+                            const int m = q0 + chalf * C::kCW + j;
                             if (m < p.M)
                                 p.y[int64_t(m) * p.ldy + n] =
                                     uint16_t(ptx::pack_bf16x2(acc[j], 0.0f) & 0xFFFF);
@@ -388,7 +430,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     if (n < p.N) {
 #pragma unroll
                         for (int j = 0; j < C::kCW; ++j) {
-                            const int m = q0 + j;
+                            const int m = q0 + chalf * C::kCW + j;
                             if (m < p.M) wsp[int64_t(m) * p.ldw + n] = acc[j];
                         }
                     }
@@ -397,11 +439,14 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         }
     }
 
+    __syncwarp();
     ptx::tc_fence_before();
-    __syncthreads();
+    if (PAIR) ptx::cluster_sync();      // both CTAs done with TMEM and with each other's barriers
+    else __syncthreads();
     if (warp == 1) {
         ptx::tc_fence_after();
-        ptx::tmem_dealloc(tmem_base, C::kTmemCols);
+        if (PAIR) ptx::tmem_dealloc_pair(tmem_base, C::kTmemCols);
+        else ptx::tmem_dealloc(tmem_base, C::kTmemCols);
     }
 }
 

@@ -1,5 +1,6 @@
 // Thin inline-PTX wrappers for the sm_100a features the GEMM uses:
-// mbarriers, TMA tiled loads (no multicast), tcgen05 MMA / TMEM.
+// mbarriers, TMA tiled loads (every CTA loads only its own tiles), cluster
+// barriers and mapa, tcgen05 MMA / TMEM for one CTA or a CTA pair.
 // Every wait is bounded: it gives up after a clock budget and reports
 // failure to the caller instead of spinning forever.
 #pragma once
@@ -52,6 +53,57 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// ----------------------------------------------------------------- cluster
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t num_clusters_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+// All threads of all CTAs of the cluster (release / acquire at cluster scope).
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Shared::cluster address of the same shared variable in CTA `rank`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+    return r;
+}
+// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+// Wait on a local mbarrier whose arrivals may come from the peer CTA.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
+                                                  long long budget = kWaitBudgetCycles) {
+    if (mbar_try_wait_cluster(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+        if (mbar_try_wait_cluster(bar, parity)) return true;
+        if (clock64() - t0 > budget) return false;
+    }
+}
+
 // ----------------------------------------------------------------- TMA
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(m)) : "memory");
@@ -70,6 +122,19 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, uin
         : "memory");
 }
 
+// 2-D tiled load for a CTA pair (cta_group::2): the data lands in this
+// CTA's shared memory, the transaction bytes complete on the mbarrier at
+// `bar_cluster` (a shared::cluster address, here the leader CTA's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m, uint32_t bar_cluster,
+                                                 int32_t c0, int32_t c1) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4}], [%2];"
+        :: "r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster),
+           "r"(c0), "r"(c1)
+        : "memory");
+}
+
 // ----------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -80,6 +145,17 @@ __device__ __forceinline__ void tmem_relinquish() {
 }
 __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
+}
+// CTA-pair versions: the same warp of both CTAs of the pair executes them.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :: "r"(smem_u32(dst_smem)), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(taddr), "r"(ncols) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -96,6 +172,25 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
         :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// CTA-pair MMA (issued by the leader CTA only): A rows 0-127 and B rows
+// 0-(N/2-1) come from the leader's shared memory, the rest from the peer's
+// at the same offsets; each CTA's TMEM receives its 128 rows of D.
+__device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
+}
+
+// Arrive once on the mbarrier at shared::cluster address `bar_cluster`
+// (this CTA's or the peer's) when the pair MMAs issued so far complete.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar_cluster) : "memory");
 }
 
 // Arrive once on `bar` when every MMA this thread issued so far completes.
@@ -176,12 +271,12 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor: E4M3 x E4M3 -> fp32, both operands K-major,
-// M = 128, N = n.
-__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n) {
+// M = m (128 for one CTA, 256 for a CTA pair), N = n.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int n, int m = 128) {
     return (1u << 4)                       // D format fp32
          | (0u << 7) | (0u << 10)          // A, B: E4M3
          | (uint32_t(n >> 3) << 17)        // N / 8
-         | (uint32_t(128 >> 4) << 24);     // M / 16
+         | (uint32_t(m >> 4) << 24);       // M / 16
 }
 
 // Two independent IEEE fp32 fused multiply-adds, a = p * s + a, per lane
@@ -194,6 +289,24 @@ __device__ __forceinline__ void fma2(float& a0, float& a1, float p0, float p1, f
         "fma.rn.f32x2 ra, rp, rs, ra;\n\t"
         "mov.b64 {%0, %1}, ra;\n\t}"
         : "+f"(a0), "+f"(a1) : "f"(p0), "f"(p1), "f"(s0), "f"(s1));
+}
+
+// Packed pair of fp32 values in one 64-bit register (low word = element 0).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+// acc = p * s + acc on a packed pair, p given as two fp32 registers.
+__device__ __forceinline__ void fma2p(uint64_t& acc, float p0, float p1, uint64_t s2) {
+    asm("{\n\t.reg .b64 rp;\n\t"
+        "mov.b64 rp, {%1, %2};\n\t"
+        "fma.rn.f32x2 %0, rp, %3, %0;\n\t}"
+        : "+l"(acc) : "f"(p0), "f"(p1), "l"(s2));
 }
 
 // Register-file split between warpgroups (all warps of a warpgroup run it).

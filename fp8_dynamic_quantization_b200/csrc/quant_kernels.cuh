@@ -38,21 +38,25 @@ __device__ __forceinline__ int64_t vec_offset(int64_t i, int64_t vec_per_row, in
 }
 
 // ---------------------------------------------------------------------------
-// Per-1x128-group quantisation.  16 threads own one group (16 x 8 values);
-// each thread carries U groups per iteration so U loads are in flight.
+// Per-1x128-group quantisation.  8 threads own one group: thread `sub`
+// holds its 16-byte chunks sub and sub+8 (16 values), so one load
+// instruction of a warp covers four 128-byte runs, fully coalesced, and the
+// per-group work (3 shuffles, the scale and its reciprocal) is shared by 16
+// values per thread.  Each thread carries U groups per iteration (2U loads
+// in flight).
 // ---------------------------------------------------------------------------
 template <int U, bool CONTIG>
 __global__ void __launch_bounds__(kQuantThreads)
 group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                       uint8_t* __restrict__ q, int64_t ldq,
                       float* __restrict__ scales, int64_t groups, int64_t G) {
-    const int sub = threadIdx.x & 15;
-    const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 4;
-    const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 4;
-    // The two halves of a warp own groups 2w and 2w+1 (g_stride is even), so
-    // testing the even one keeps the loop warp-uniform for the shuffles.
-    for (int64_t g0 = g_first; (g0 & ~int64_t(1)) < groups; g0 += U * g_stride) {
-        uint4 v[U];
+    const int sub = threadIdx.x & 7;
+    const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 3;
+    const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 3;
+    // A warp owns groups 4w..4w+3 (g_stride is a multiple of 4), so testing
+    // the first of them keeps the loop warp-uniform for the shuffles.
+    for (int64_t g0 = g_first; (g0 & ~int64_t(3)) < groups; g0 += U * g_stride) {
+        uint4 a[U], b[U];
         int64_t xo[U], qo[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -65,19 +69,21 @@ group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                 xo[u] = r * ldx + c * 128 + sub * 8;
                 qo[u] = r * ldq + c * 128 + sub * 8;
             }
-            v[u] = (g < groups) ? ld_stream16(x + xo[u]) : make_uint4(0, 0, 0, 0);
+            const bool ok = g < groups;
+            a[u] = ok ? ld_stream16(x + xo[u]) : make_uint4(0, 0, 0, 0);
+            b[u] = ok ? ld_stream16(x + xo[u] + 64) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t g = g0 + u * g_stride;
-            uint32_t m = absmax8(v[u]);
-            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 8));
+            uint32_t m = max(absmax8(a[u]), absmax8(b[u]));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
+            const Scale d = make_scale(scale_from_amax_bits(m));
             if (g < groups) {
-                st_stream8(q + qo[u], quant8(v[u], d));
+                st_stream8(q + qo[u], quant8(a[u], d));
+                st_stream8(q + qo[u] + 64, quant8(b[u], d));
                 if (sub == 0) scales[g] = d.s;
             }
         }
@@ -124,7 +130,7 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
     for (int i = threadIdx.x; i < nparts; i += kQuantThreads)
         m = max(m, __ldcg(partials + i) & 0x7FFFu);
     m = block_max<kQuantThreads>(m, red);
-    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
+    const Scale d = make_scale(scale_from_amax_bits(m));
     if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = d.s;
 
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
@@ -152,26 +158,46 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
 }
 
 // ---------------------------------------------------------------------------
-// Per-tensor, single launch, for tensors that fit in the registers of one
-// co-resident grid (cooperative launch).  Barrier state lives in the
-// caller's workspace: ws[0] arrival count, ws[1] generation, ws[2..] one
-// partial max per CTA.  The last CTA to arrive resets the count and bumps
-// the generation; the others wait for the generation to change, at most
-// `spin_limit` polls, after which they record FP8Q_ERR_TIMEOUT and return
-// without writing outputs.
+// Per-tensor, single launch, for tensors that fit in the registers of a grid
+// of at most one CTA per SM (all CTAs resident together).  Barrier state
+// lives in the caller's workspace: ws[0] arrival count, ws[1] = generation
+// (high 16 bits) | amax (low 16 bits), ws[2..] one partial max per CTA.
+// Every CTA publishes its partial and arrives (acq_rel atomic); the last one
+// reduces the partials, resets the count and publishes generation+1 with
+// the amax (release); the others poll ws[1] (acquire), at most `spin_limit`
+// polls, after which they record FP8Q_ERR_TIMEOUT and return without
+// writing outputs.  A one-CTA grid needs no barrier at all.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+    return old;
+}
+__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.gpu.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
 template <int U, bool CONTIG>
 __global__ void __launch_bounds__(kQuantThreads)
 per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
                         int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                         float* __restrict__ scale_out, uint32_t* ws, int64_t spin_limit) {
     __shared__ uint32_t red[kQuantThreads / 32];
-    __shared__ int s_ok;
+    __shared__ uint32_t s_word;     // bit 31: timed out; bit 30: this CTA is last; low 16: amax
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
     const int64_t first = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
-    volatile uint32_t* vws = ws;
     uint32_t gen0 = 0;
-    if (threadIdx.x == 0) gen0 = vws[1];
+    if (gridDim.x > 1 && threadIdx.x == 0) gen0 = ld_relaxed_gpu(ws + 1) >> 16;
 
     uint4 v[U];
 #pragma unroll
@@ -185,32 +211,45 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
     for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
     m = block_max<kQuantThreads>(m, red);
 
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        ws[2 + blockIdx.x] = m;
-        __threadfence();
-        const uint32_t arrived = atomicAdd(ws, 1u);
-        if (arrived == gridDim.x - 1) {
-            ws[0] = 0;
-            __threadfence();
-            atomicAdd(ws + 1, 1u);
-        } else {
-            int64_t n = 0;
-            while (vws[1] == gen0) {
-                if (++n > spin_limit) { ok = 0; record_error(6 /* FP8Q_ERR_TIMEOUT */); break; }
-                __nanosleep(32);
+    uint32_t amax = m;
+    if (gridDim.x > 1) {
+        if (threadIdx.x == 0) {
+            ws[2 + blockIdx.x] = m;
+            const uint32_t arrived = atom_add_acq_rel_gpu(ws, 1u);
+            uint32_t word = 0;
+            if (arrived == gridDim.x - 1) {
+                word = 1u << 30;
+            } else {
+                int64_t n = 0;
+                uint32_t w1;
+                while (((w1 = ld_acquire_gpu(ws + 1)) >> 16) == gen0) {
+                    if (++n > spin_limit) break;
+                    __nanosleep(20);
+                }
+                word = ((w1 >> 16) == gen0) ? (1u << 31) : (w1 & 0xFFFFu);
+                if (word >> 31) record_error(6 /* FP8Q_ERR_TIMEOUT */);
             }
+            s_word = word;
         }
-        __threadfence();
-        s_ok = ok;
+        __syncthreads();
+        const uint32_t word = s_word;
+        if (word >> 31) return;
+        if (word & (1u << 30)) {
+            // last CTA: reduce the partials, reset the count, publish
+            uint32_t mm = 0;
+            for (int i = threadIdx.x; i < int(gridDim.x); i += kQuantThreads)
+                mm = max(mm, ld_relaxed_gpu(ws + 2 + i));
+            mm = block_max<kQuantThreads>(mm, red);
+            if (threadIdx.x == 0) {
+                ws[0] = 0;
+                st_release_gpu(ws + 1, (((gen0 + 1) & 0xFFFFu) << 16) | mm);
+            }
+            amax = mm;
+        } else {
+            amax = word & 0xFFFFu;
+        }
     }
-    __syncthreads();
-    if (!s_ok) return;
-
-    uint32_t mm = 0;
-    for (int i = threadIdx.x; i < int(gridDim.x); i += kQuantThreads) mm = max(mm, __ldcg(ws + 2 + i));
-    mm = block_max<kQuantThreads>(mm, red);
-    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(mm)));
+    const Scale d = make_scale(scale_from_amax_bits(amax));
     if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = d.s;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
@@ -234,7 +273,7 @@ reduce_partials_kernel(const uint32_t* __restrict__ partials, int n, uint32_t* _
 
 // scale = amax / 448 from an amax word, for an empty apply.
 __global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float* __restrict__ scale) {
-    if (threadIdx.x == 0) *scale = scale_from_amax(amax_bits_to_f32(*amax_bits));
+    if (threadIdx.x == 0) *scale = scale_from_amax_bits(*amax_bits & 0x7FFFu);
 }
 
 // ---------------------------------------------------------------------------
@@ -258,7 +297,7 @@ block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
         m = max(m, absmax8(v[u]));
     }
     m = block_max<kQuantThreads>(m, red);
-    const Scale d = make_scale(scale_from_amax(amax_bits_to_f32(m)));
+    const Scale d = make_scale(scale_from_amax_bits(m));
     if (threadIdx.x == 0) sb[nb * G + kb] = d.s;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {

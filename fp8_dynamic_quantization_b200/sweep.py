@@ -6,7 +6,8 @@
 
 Every measurement is the median over `reps` of one call, timed with CUDA
 events on the launching stream.  Mode "cold": an L2 flush (a 256 MB write)
-runs before every call and is outside the timed interval.  Mode "graph":
+and a ~100 us GPU sleep run before every call, outside the timed interval
+(the sleep hides the host's launch overhead).  Mode "graph":
 `reps` calls captured in one CUDA graph and replayed; time / reps (this is how
 the pages timed their amax kernel; inputs that fit in L2 stay L2-warm).
 One JSON line per measurement: op, shape, microseconds, algorithmic GB/s
@@ -46,6 +47,9 @@ class Timer:
         ts = []
         for _ in range(reps):
             self.flush_buf.fill_(1)
+            # keep the GPU busy while the host prepares the call, so host-side
+            # overhead never shows up between the two events
+            torch.cuda._sleep(200_000)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record()
             fn()

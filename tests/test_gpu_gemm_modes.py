@@ -1,0 +1,40 @@
+"""Every GEMM launch mode against the oracle, forced through the tuning
+override FP8Q_GEMM_TILE (read once per process, hence one child process per
+mode).  The default launch table only selects some of them."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+CHILD = r'''
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import oracle
+import fp8_dynamic_quantization_b200 as fq
+from fp8_dynamic_quantization_b200 import inputs
+dev = torch.device("cuda:0")
+for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 256)]:
+    qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m + n + k)
+    y = fq.block_gemm(torch.from_numpy(qa).to(dev), torch.from_numpy(sa).to(dev),
+                      torch.from_numpy(qb).to(dev), torch.from_numpy(sb).to(dev))
+    R, T = oracle.block_gemm(qa, sa, qb, sb)
+    Y = y.float().cpu().numpy().astype(np.float64)
+    bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
+    assert bad == 0, (m, n, k, bad)
+assert fq.device_status() == 0
+print("ok")
+'''
+
+
+@pytest.mark.parametrize("tile", ["normal:128", "normal:192", "normal:256", "pair:256", "pair:128",
+                                  "swap:16", "swap:64", "swap:128:3"])
+def test_gemm_mode_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
+    env = dict(os.environ, FP8Q_GEMM_TILE=tile)
+    r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
