@@ -64,6 +64,35 @@ def bytes_gemm(m, n, k=K):
     return m * k + n * k + 4.0 * m * g + 4.0 * ((n + 127) // 128) * g + 2.0 * m * n
 
 
+GEMM_SOURCES = ("gemm_kernels.cuh", "ptx_sm100.cuh", "launch_table.inc")
+TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "block_gemm_prefill_4096xNx7168.md")
+
+
+def gemm_traffic():
+    """DRAM bytes per GEMM launch (mean over the step's three launches) from
+    the committed ncu summary -- only while the GEMM sources still hash to the
+    value recorded there; None otherwise."""
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fp8_dynamic_quantization_b200", "csrc")
+    try:
+        for f in GEMM_SOURCES:
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(fh.read())
+        rec = {}
+        with open(TRAFFIC_RECORD) as fh:
+            for line in fh:
+                if ":" in line and line.split(":", 1)[0].strip() in (
+                        "gemm_source_sha256_16", "dram_bytes_per_launch_mean"):
+                    k, v = line.split(":", 1)
+                    rec[k.strip()] = v.split()[0]
+    except OSError:
+        return None
+    if rec.get("gemm_source_sha256_16") != h.hexdigest()[:16]:
+        return None
+    return float(rec["dram_bytes_per_launch_mean"])
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -333,7 +362,9 @@ def our_arm(args, rank, world, local_rank):
             "kernels": kernels,
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak,
                          "unit": "TFLOP/s", "frac": achieved / fp8_peak,
-                         "traffic": None,
+                         "traffic": gemm_traffic(),
+                         "traffic_unit": "bytes per GEMM launch (mean of the step's 3), ncu",
+                         "algorithmic_bytes_per_launch": sum(bytes_gemm(M, n) for n in NS) / len(NS),
                          "kernel": "block_gemm_kernel (all three N per step)",
                          "peak_source": f"{peak_src} bf16 "
                                         f"{'burst' if timed_s < 5.0 else 'sustained'} x {FP8_OVER_BF16} (fp8/bf16 nominal)"},

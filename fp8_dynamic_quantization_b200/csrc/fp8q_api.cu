@@ -360,7 +360,7 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
     // are resident together, so the grid barrier completes; it is bounded
     // anyway and reports FP8Q_ERR_TIMEOUT instead of hanging).
     if (fused_grid <= std::min<int64_t>(std::min(d->fused_capacity, d->sms), kMaxPartials)) {
-        const int64_t spin = int64_t(1) << 24;
+        const int64_t spin = int64_t(2000000000);     // ~1 s of SM clock
         const uint16_t* xs = static_cast<const uint16_t*>(x);
         if (log_enabled())
             std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: fused grid=%lld\n",

@@ -164,9 +164,9 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
 // (high 16 bits) | amax (low 16 bits), ws[2..] one partial max per CTA.
 // Every CTA publishes its partial and arrives (acq_rel atomic); the last one
 // reduces the partials, resets the count and publishes generation+1 with
-// the amax (release); the others poll ws[1] (acquire), at most `spin_limit`
-// polls, after which they record FP8Q_ERR_TIMEOUT and return without
-// writing outputs.  A one-CTA grid needs no barrier at all.
+// the amax (release); the others poll ws[1] (acquire) for at most
+// `spin_cycles` SM clock cycles, after which they record FP8Q_ERR_TIMEOUT and
+// return without writing outputs.  A one-CTA grid needs no barrier at all.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
     uint32_t old;
@@ -191,7 +191,7 @@ template <int U, bool CONTIG>
 __global__ void __launch_bounds__(kQuantThreads)
 per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
                         int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
-                        float* __restrict__ scale_out, uint32_t* ws, int64_t spin_limit) {
+                        float* __restrict__ scale_out, uint32_t* ws, int64_t spin_cycles) {
     __shared__ uint32_t red[kQuantThreads / 32];
     __shared__ uint32_t s_word;     // bit 31: timed out; bit 30: this CTA is last; low 16: amax
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
@@ -220,10 +220,10 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
             if (arrived == gridDim.x - 1) {
                 word = 1u << 30;
             } else {
-                int64_t n = 0;
+                const long long t0 = clock64();
                 uint32_t w1;
                 while (((w1 = ld_acquire_gpu(ws + 1)) >> 16) == gen0) {
-                    if (++n > spin_limit) break;
+                    if (clock64() - t0 > spin_cycles) break;
                     __nanosleep(20);
                 }
                 word = ((w1 >> 16) == gen0) ? (1u << 31) : (w1 & 0xFFFFu);
