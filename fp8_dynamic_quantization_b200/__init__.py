@@ -77,7 +77,7 @@ def act_quant_per_tensor(x: torch.Tensor):
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     s = torch.empty(1, dtype=torch.float32, device=x.device)
     nbytes = lib.fp8_act_quant_per_tensor_workspace_size(M, K)
-    ws = _workspace("per_tensor", x.device, nbytes, zero=True)
+    ws = _workspace("per_tensor", x.device, nbytes, zero=False)
     _abi.check(lib.fp8_act_quant_per_tensor(x.data_ptr(), M, K, ldx, q.data_ptr(), K, s.data_ptr(),
                                             ws.data_ptr(), ws.numel(), _stream(x.device)),
                "fp8_act_quant_per_tensor")

@@ -41,14 +41,13 @@ struct DeviceInfo {
     bool ready = false;
     int status = FP8Q_OK;
     int sms = 0;
-    int fused_capacity = 0;   // co-resident CTAs of the fused per-tensor kernel
 };
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
 
-constexpr int kFusedU = 8;          // vectors per thread in the fused kernel
+constexpr int kClusterU = 8;        // vectors per thread in the one-cluster per-tensor kernel
 constexpr int kStreamU = 4;         // vectors per thread per iteration elsewhere
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
@@ -80,17 +79,6 @@ int device_info(DeviceInfo** out) {
             d.status = FP8Q_OK;
             if (prop.major != 10) d.status = FP8Q_ERR_NO_DEVICE;
             d.sms = prop.multiProcessorCount;
-            int per_sm = 0;
-            if (d.status == FP8Q_OK &&
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &per_sm, per_tensor_fused_kernel<kFusedU, true>, kQuantThreads, 0) != cudaSuccess)
-                d.status = FP8Q_ERR_CUDA;
-            int per_sm_nc = 0;
-            if (d.status == FP8Q_OK &&
-                cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-                    &per_sm_nc, per_tensor_fused_kernel<kFusedU, false>, kQuantThreads, 0) != cudaSuccess)
-                d.status = FP8Q_ERR_CUDA;
-            d.fused_capacity = std::min(per_sm, per_sm_nc) * d.sms;
             if (d.status == FP8Q_OK) {
                 cudaError_t e = cudaSuccess;
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12>();
@@ -154,6 +142,32 @@ struct GemmPlan {
     int64_t ldw;
     size_t ws_bytes;
 };
+
+// Measurement override: FP8Q_PER_TENSOR_PATH=twopass makes every per-tensor
+// call take the amax + apply passes (same result).
+bool per_tensor_two_pass_forced() {
+    static const bool v = [] {
+        const char* e = std::getenv("FP8Q_PER_TENSOR_PATH");
+        return e && std::strcmp(e, "twopass") == 0;
+    }();
+    return v;
+}
+
+// Bound on every barrier wait inside the GEMM, in SM clock cycles (about
+// two seconds by default).  FP8Q_WAIT_BUDGET_CYCLES overrides it for fault
+// testing; it never changes the result of a call that completes.
+long long wait_budget_cycles() {
+    static const long long v = [] {
+        const char* e = std::getenv("FP8Q_WAIT_BUDGET_CYCLES");
+        if (e && e[0]) {
+            char* end = nullptr;
+            const long long b = std::strtoll(e, &end, 10);
+            if (end && *end == 0 && b >= 0) return b;
+        }
+        return 4000000000LL;
+    }();
+    return v;
+}
 
 // Tuning override of the table (FP8Q_GEMM_TILE="normal:128", "swap:64:4",
 // ...: mode, tile width, optional split-K count).  For measuring launch
@@ -354,27 +368,38 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
     const int64_t vpr = K / 8, nvec = M * vpr;
     const bool contig = (ldx == K && ldq == K);
     uint32_t* ws = static_cast<uint32_t*>(workspace);
-    const int64_t fused_grid = (nvec + int64_t(kQuantThreads) * kFusedU - 1) /
-                               (int64_t(kQuantThreads) * kFusedU);
-    // Single launch when every CTA fits on its own SM at once (all of them
-    // are resident together, so the grid barrier completes; it is bounded
-    // anyway and reports FP8Q_ERR_TIMEOUT instead of hanging).
-    if (fused_grid <= std::min<int64_t>(std::min(d->fused_capacity, d->sms), kMaxPartials)) {
-        const int64_t spin = int64_t(2000000000);     // ~1 s of SM clock
-        const uint16_t* xs = static_cast<const uint16_t*>(x);
+    // Single launch when the tensor fits in the registers of one cluster of
+    // up to 8 CTAs; the partial maxima are exchanged through distributed
+    // shared memory.
+    constexpr int kClusterThreads = 256;
+    const int64_t per_cta = int64_t(kClusterThreads) * kClusterU;
+    const int64_t csize = (nvec + per_cta - 1) / per_cta;
+    if (csize <= kClusterMax && !per_tensor_two_pass_forced()) {
         if (log_enabled())
-            std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: fused grid=%lld\n",
-                         (long long)M, (long long)K, (long long)fused_grid);
-        if (contig)
-            per_tensor_fused_kernel<kFusedU, true><<<unsigned(fused_grid), kQuantThreads, 0, st>>>(
-                xs, nvec, vpr, ldx, q, ldq, scale, ws, spin);
-        else
-            per_tensor_fused_kernel<kFusedU, false><<<unsigned(fused_grid), kQuantThreads, 0, st>>>(
-                xs, nvec, vpr, ldx, q, ldq, scale, ws, spin);
+            std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: one cluster of %lld CTAs\n",
+                         (long long)M, (long long)K, (long long)csize);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(unsigned(csize));
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = unsigned(csize);
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = csize > 1 ? 1 : 0;        // one CTA: a plain launch
+        const uint16_t* xs = static_cast<const uint16_t*>(x);
+        const cudaError_t e =
+            contig ? cudaLaunchKernelEx(&cfg, per_tensor_cluster_kernel<kClusterU, true, kClusterThreads>, xs,
+                                        nvec, vpr, ldx, q, ldq, scale)
+                   : cudaLaunchKernelEx(&cfg, per_tensor_cluster_kernel<kClusterU, false, kClusterThreads>, xs,
+                                        nvec, vpr, ldx, q, ldq, scale);
+        if (e != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
         return launch_status(1);
     }
     const int grid = stream_grid(nvec, d->sms);
-    uint32_t* partials = ws + 2;
+    uint32_t* partials = ws;
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: amax+apply grid=%d\n",
                      (long long)M, (long long)K, grid);
@@ -549,6 +574,7 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
     p.splits = pl.splits;
     p.units = pl.units;
     p.scale_vec4 = (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
+    p.wait_budget = wait_budget_cycles();
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
                      (long long)M, (long long)N, (long long)K,

@@ -53,6 +53,7 @@ struct GemmParams {
     int M, N, G;
     int tiles_p, tiles_q, splits, units;
     int scale_vec4;      // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
+    long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 
 template <int BN, bool SWAP, int STAGES, bool PAIR = false>
@@ -203,7 +204,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1)) { fail(); break; }
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, p.wait_budget)) { fail(); break; }
                     uint8_t* dst = tiles + size_t(s) * C::kStageBytes;
                     if (PAIR) {
                         // both CTAs' copies complete on the leader's barrier
@@ -235,10 +236,10 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
                     const uint32_t buf = c % NB, tph = (c / NB) & 1;
-                    const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1)
-                                            : ptx::mbar_wait(&tempty[buf], tph ^ 1);
+                    const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1, p.wait_budget)
+                                            : ptx::mbar_wait(&tempty[buf], tph ^ 1, p.wait_budget);
                     if (!freed) { fail(); break; }
-                    if (!ptx::mbar_wait(&full[s], ph)) { fail(); break; }
+                    if (!ptx::mbar_wait(&full[s], ph, p.wait_budget)) { fail(); break; }
                     ptx::tc_fence_after();
                     const uint32_t pa = ptx::smem_u32(tiles + size_t(s) * C::kStageBytes);
                     const uint32_t qa = pa + C::kPBytes;
@@ -333,7 +334,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 }
                 const uint64_t s2 = ptx::pack_f32x2(s, s);
                 const uint32_t buf = c % NB, tph = (c / NB) & 1;
-                if (!ptx::mbar_wait(&tfull[buf], tph)) { fail(); ok = false; break; }
+                if (!ptx::mbar_wait(&tfull[buf], tph, p.wait_budget)) { fail(); ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16)
                                        + buf * BN + chalf * C::kCW;

@@ -16,8 +16,9 @@
 //                            writes codes.  Walks the tensor backwards, so
 //                            the part of x the amax pass read last is still
 //                            in L2 when it is read again.
-//  per_tensor_fused_kernel   small tensors: one launch; values stay in
-//                            registers across a bounded grid barrier.
+//  per_tensor_cluster_kernel small tensors: one launch of one thread-block
+//                            cluster; values stay in registers while the
+//                            CTAs exchange partial maxima on chip.
 //  block128_quant_kernel     128x128 weight blocks (offline step).
 #pragma once
 
@@ -158,46 +159,44 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
 }
 
 // ---------------------------------------------------------------------------
-// Per-tensor, single launch, for tensors that fit in the registers of a grid
-// of at most one CTA per SM (all CTAs resident together).  Barrier state
-// lives in the caller's workspace: ws[0] arrival count, ws[1] = generation
-// (high 16 bits) | amax (low 16 bits), ws[2..] one partial max per CTA.
-// Every CTA publishes its partial and arrives (acq_rel atomic); the last one
-// reduces the partials, resets the count and publishes generation+1 with
-// the amax (release); the others poll ws[1] (acquire) for at most
-// `spin_cycles` SM clock cycles, after which they record FP8Q_ERR_TIMEOUT and
-// return without writing outputs.  A one-CTA grid needs no barrier at all.
+// Per-tensor, single launch, for tensors that fit in the registers of one
+// thread-block cluster (up to 8 CTAs of NT threads, U vectors per thread;
+// a single CTA is launched without a cluster and needs no exchange).  Each CTA reduces its values to one partial max in shared
+// memory; after a cluster barrier every CTA reads all partials through
+// distributed shared memory (mapa + ld.shared::cluster), so the whole amax
+// exchange stays on chip.  A second barrier phase keeps each CTA's shared
+// memory alive until every peer has read it.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
-    uint32_t old;
-    asm volatile("atom.add.acq_rel.gpu.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
-    return old;
+constexpr int kClusterMax = 8;
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
 }
-__device__ __forceinline__ void st_release_gpu(uint32_t* p, uint32_t v) {
-    asm volatile("st.release.gpu.u32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
 }
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint32_t ld_shared_cluster(const uint32_t* local, uint32_t rank) {
+    uint32_t addr = static_cast<uint32_t>(__cvta_generic_to_shared(local)), remote, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(addr), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(remote) : "memory");
     return v;
 }
 
-template <int U, bool CONTIG>
-__global__ void __launch_bounds__(kQuantThreads)
-per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
-                        int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
-                        float* __restrict__ scale_out, uint32_t* ws, int64_t spin_cycles) {
-    __shared__ uint32_t red[kQuantThreads / 32];
-    __shared__ uint32_t s_word;     // bit 31: timed out; bit 30: this CTA is last; low 16: amax
-    const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
-    const int64_t first = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
-    uint32_t gen0 = 0;
-    if (gridDim.x > 1 && threadIdx.x == 0) gen0 = ld_relaxed_gpu(ws + 1) >> 16;
+template <int U, bool CONTIG, int NT>
+__global__ void __launch_bounds__(NT)
+per_tensor_cluster_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
+                          int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
+                          float* __restrict__ scale_out) {
+    constexpr int kClusterThreads = NT;
+    __shared__ uint32_t red[kClusterThreads / 32];
+    __shared__ uint32_t part;                     // this CTA's partial max
+    const uint32_t crank = cluster_rank(), csize = cluster_nctarank();
+    const int64_t stride = int64_t(csize) * kClusterThreads;
+    const int64_t first = int64_t(crank) * kClusterThreads + threadIdx.x;
 
     uint4 v[U];
 #pragma unroll
@@ -209,48 +208,21 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
     uint32_t m = 0;
 #pragma unroll
     for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
-    m = block_max<kQuantThreads>(m, red);
-
-    uint32_t amax = m;
-    if (gridDim.x > 1) {
-        if (threadIdx.x == 0) {
-            ws[2 + blockIdx.x] = m;
-            const uint32_t arrived = atom_add_acq_rel_gpu(ws, 1u);
-            uint32_t word = 0;
-            if (arrived == gridDim.x - 1) {
-                word = 1u << 30;
-            } else {
-                const long long t0 = clock64();
-                uint32_t w1;
-                while (((w1 = ld_acquire_gpu(ws + 1)) >> 16) == gen0) {
-                    if (clock64() - t0 > spin_cycles) break;
-                    __nanosleep(20);
-                }
-                word = ((w1 >> 16) == gen0) ? (1u << 31) : (w1 & 0xFFFFu);
-                if (word >> 31) record_error(6 /* FP8Q_ERR_TIMEOUT */);
-            }
-            s_word = word;
-        }
-        __syncthreads();
-        const uint32_t word = s_word;
-        if (word >> 31) return;
-        if (word & (1u << 30)) {
-            // last CTA: reduce the partials, reset the count, publish
-            uint32_t mm = 0;
-            for (int i = threadIdx.x; i < int(gridDim.x); i += kQuantThreads)
-                mm = max(mm, ld_relaxed_gpu(ws + 2 + i));
-            mm = block_max<kQuantThreads>(mm, red);
-            if (threadIdx.x == 0) {
-                ws[0] = 0;
-                st_release_gpu(ws + 1, (((gen0 + 1) & 0xFFFFu) << 16) | mm);
-            }
-            amax = mm;
-        } else {
-            amax = word & 0xFFFFu;
-        }
+    m = block_max<kClusterThreads>(m, red);
+    if (threadIdx.x == 0) part = m;
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    uint32_t mm = 0;
+    if (threadIdx.x < 32) {
+        if (threadIdx.x < csize) mm = ld_shared_cluster(&part, threadIdx.x);
+        mm = warp_max(mm);
     }
-    const Scale d = make_scale(scale_from_amax_bits(amax));
-    if (blockIdx.x == 0 && threadIdx.x == 0) *scale_out = d.s;
+    // done reading the peers' shared memory
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    if (threadIdx.x == 0) red[0] = mm;
+    __syncthreads();
+    const Scale d = make_scale(scale_from_amax_bits(red[0]));
+    if (crank == 0 && threadIdx.x == 0) *scale_out = d.s;
 #pragma unroll
     for (int u = 0; u < U; ++u) {
         const int64_t i = first + u * stride;
@@ -259,6 +231,8 @@ per_tensor_fused_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t ve
             st_stream8(q + qo, quant8(v[u], d));
         }
     }
+    // keep this CTA's shared memory until every peer has read it
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
 // out = max(partials[0:n]); one CTA.

@@ -50,7 +50,11 @@
  *   - Determinism: the same inputs give the same bytes, whatever the
  *     launch configuration chosen.
  *   - Environment: FP8Q_LOG=1 prints the launch chosen for every call to
- *     stderr.  No environment variable changes numerics.
+ *     stderr.  FP8Q_GEMM_TILE forces a GEMM launch mode and
+ *     FP8Q_PER_TENSOR_PATH=twopass the two-pass per-tensor path (measurement);
+ *     FP8Q_WAIT_BUDGET_CYCLES bounds the GEMM's device-side waits (fault
+ *     testing); both are read once per process.  No environment variable
+ *     changes the result of a call that completes.
  */
 #ifndef FP8Q_H
 #define FP8Q_H
@@ -85,17 +89,16 @@ int fp8q_abi_version(void);
 /* ------------------------------------------------------------------ */
 
 /* Bytes of device workspace fp8_act_quant_per_tensor needs for an [M,K]
- * input on the current device.  The workspace must be ZERO-FILLED before
- * its first use; every completed call leaves it ready for the next call.
- * Calls sharing one workspace must be ordered (same stream, or joined).
- * After FP8Q_ERR_TIMEOUT the caller must zero it again. */
+ * input (partial maxima of the amax pass; no zero fill needed).  Calls
+ * sharing one workspace must be ordered (same stream, or joined). */
 size_t fp8_act_quant_per_tensor_workspace_size(int64_t M, int64_t K);
 
 /* x: bf16 [M,K], row stride ldx.  Writes codes q: uint8 [M,K], row stride
  * ldq, and *scale (one fp32 on the device) = fl32(amax / 448), with
  * amax = max |x| over the whole tensor (exact).  K must be a multiple of 8.
- * M == 0 or K == 0 writes scale 0 and nothing else.  Small tensors (one
- * CTA per SM suffices) take a single launch with a bounded grid barrier;
+ * M == 0 or K == 0 writes scale 0 and nothing else.  Tensors of up to
+ * 128K elements take a single launch of one thread-block cluster (up to 8
+ * CTAs exchange their partial maxima through distributed shared memory);
  * larger ones take an amax pass with an input-sized grid and then an apply
  * pass that re-reads x in reverse order (its tail is still in L2). */
 int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx,

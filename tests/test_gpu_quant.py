@@ -127,7 +127,7 @@ def test_per_tensor_other_shapes(oracle_mod, gpu, m, k):
 
 
 def test_per_tensor_repeated_calls_reuse_workspace(oracle_mod, gpu):
-    """The fused path's barrier state resets itself between calls."""
+    """Back-to-back calls of both paths (one cluster, two passes) with one cached workspace."""
     for m in (64, 1024, 1, 300, 65536, 256, 64):
         x = inputs.activations_per_tensor(m, seed=77 + m)
         q_ref, s_ref = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
