@@ -10,6 +10,7 @@ calls raise if the library is missing or the device is not sm_100.
     qb, sb = weight_quant_block128(w)     # one scale per 128x128 block
     y      = block_gemm(q, S, qb, sb)     # bf16 Y = A * B^T, block-scaled
     y      = linear(x, qb, sb)            # group quant + block GEMM
+    y      = gemm_per_tensor(q, s, qw, sw)  # per-tensor scales: Y = s*sw*A*B^T
 
 Codes are returned as ``torch.float8_e4m3fn`` tensors, scales as float32.
 """
@@ -23,7 +24,8 @@ from . import _abi
 
 __all__ = [
     "act_quant_per_tensor", "act_amax", "act_quant_apply", "act_quant_group128",
-    "weight_quant_block128", "block_gemm", "linear", "device_status",
+    "weight_quant_block128", "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
+    "device_status",
     "per_tensor_sharded", "Fp8qError", "library",
 ]
 
@@ -174,6 +176,41 @@ def block_gemm(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.T
                                   out.data_ptr(), ldy, M, N, K, ws_ptr, ws_len, _stream(qa.device)),
                "fp8_block_gemm")
     return out
+
+
+def gemm_per_tensor(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                    out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 Y[M,N] = sa * sb * A * B^T with one fp32 scale per operand
+    (sa, sb: float32 [1] device tensors, e.g. from act_quant_per_tensor)."""
+    lib = _abi.load()
+    M, K, lda = _rows(_codes(qa, "qa"), "qa")
+    N, Kb, ldb = _rows(_codes(qb, "qb"), "qb")
+    if K != Kb:
+        raise ValueError("qa and qb must share K")
+    for t, name in ((sa, "sa"), (sb, "sb")):
+        if t.dtype != torch.float32 or t.numel() != 1 or not t.is_cuda:
+            raise ValueError(f"{name} must be a float32 [1] CUDA tensor")
+    if out is None:
+        ldy_alloc = (N + 7) // 8 * 8
+        out = torch.empty((M, ldy_alloc), dtype=torch.bfloat16, device=qa.device)[:, :N]
+    _, _, ldy = _rows(out, "out")
+    nbytes = lib.fp8_block_gemm_workspace_size(M, N, K)
+    ws_ptr, ws_len = None, 0
+    if nbytes:
+        ws = _workspace("gemm", qa.device, nbytes, zero=False)
+        ws_ptr, ws_len = ws.data_ptr(), ws.numel()
+    _abi.check(lib.fp8_gemm_per_tensor(qa.data_ptr(), lda, sa.data_ptr(), qb.data_ptr(), ldb, sb.data_ptr(),
+                                       out.data_ptr(), ldy, M, N, K, ws_ptr, ws_len, _stream(qa.device)),
+               "fp8_gemm_per_tensor")
+    return out
+
+
+def linear_per_tensor(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:
+    """The dynamic per-tensor FP8 linear method: per-tensor quantisation of x
+    (exact amax, scale = amax/448), then the per-tensor-scaled GEMM against
+    weight codes qb with scale sb."""
+    qa, sa = act_quant_per_tensor(x)
+    return gemm_per_tensor(qa, sa, qb, sb)
 
 
 def linear(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:

@@ -52,11 +52,11 @@ constexpr int kStreamU = 4;         // vectors per thread per iteration elsewher
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
 cudaError_t set_gemm_smem() {
-    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR>,
+    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(GemmCfg<BN, SWAP, STAGES, PAIR>::kSmemBytes));
+                                int(GemmCfg<BN, SWAP, STAGES, PAIR, PT>::kSmemBytes));
 }
 
 // Device facts, queried once per device.  FP8Q_ERR_NO_DEVICE unless the
@@ -90,6 +90,13 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, true>();
                 if (e != cudaSuccess) { cudaGetLastError(); d.status = FP8Q_ERR_CUDA; }
             }
             d.ready = true;
@@ -194,7 +201,9 @@ bool tile_override(TableRow* out) {
     return has;
 }
 
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
+// The per-tensor GEMM has no CTA-pair variant: a forced pair row runs as the
+// single-CTA tile of the same width.
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool per_tensor = false) {
     GemmPlan pl{};
     const TableRow* row = &kGemmTable[0];
     for (const TableRow& r : kGemmTable)
@@ -202,7 +211,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms) {
     TableRow forced;
     if (tile_override(&forced)) row = &forced;
     pl.swap = row->mode == kSwap;
-    pl.pair = row->mode == kPair;
+    pl.pair = row->mode == kPair && !per_tensor;
     pl.bn = row->bn;
     pl.stages = pl.swap ? (pl.bn == 16 ? 12 : pl.bn == 32 ? 10 : pl.bn == 64 ? 8 : 6)
                         : pl.pair ? (pl.bn == 256 ? 6 : 8) : (pl.bn == 192 ? 5 : pl.bn == 256 ? 4 : 6);
@@ -265,12 +274,12 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& p, int grid,
                  cudaStream_t st) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR>;
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT>;
     if (!PAIR) {
-        block_gemm_kernel<BN, SWAP, STAGES, PAIR><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+        block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
         return;
     }
     cudaLaunchConfig_t cfg = {};
@@ -525,9 +534,11 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
     return plan_gemm(M, N, K, d->sms).ws_bytes;
 }
 
-int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
-                   const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                   void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
+                    const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                    void* workspace, size_t workspace_bytes, void* stream, bool per_tensor) {
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
@@ -546,7 +557,7 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms);
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, per_tensor);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -573,14 +584,29 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
     p.tiles_q = pl.tiles_q;
     p.splits = pl.splits;
     p.units = pl.units;
-    p.scale_vec4 = (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
+    p.scale_vec4 = !per_tensor && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
     p.wait_budget = wait_budget_cycles();
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
-    if (pl.swap) {
+    if (per_tensor) {
+        if (pl.swap) {
+            switch (pl.bn) {
+                case 16: launch_gemm<16, true, 12, false, true>(tp, tq, p, pl.grid, st); break;
+                case 32: launch_gemm<32, true, 10, false, true>(tp, tq, p, pl.grid, st); break;
+                case 64: launch_gemm<64, true, 8, false, true>(tp, tq, p, pl.grid, st); break;
+                default: launch_gemm<128, true, 6, false, true>(tp, tq, p, pl.grid, st); break;
+            }
+        } else if (pl.bn == 128) {
+            launch_gemm<128, false, 6, false, true>(tp, tq, p, pl.grid, st);
+        } else if (pl.bn == 192) {
+            launch_gemm<192, false, 5, false, true>(tp, tq, p, pl.grid, st);
+        } else {
+            launch_gemm<256, false, 4, false, true>(tp, tq, p, pl.grid, st);
+        }
+    } else if (pl.swap) {
         switch (pl.bn) {
             case 16: launch_gemm<16, true, 12>(tp, tq, p, pl.grid, st); break;
             case 32: launch_gemm<32, true, 10>(tp, tq, p, pl.grid, st); break;
@@ -603,6 +629,20 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_
         rc = launch_status();
     }
     return rc;
+}
+
+extern "C" {
+
+int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
+                   const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, false);
+}
+
+int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
+                        const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, true);
 }
 
 // ------------------------------------------------------------ GEMM, no allocation

@@ -36,6 +36,11 @@
 //           is computed once per work unit into shared memory.
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
+//
+// PT (per-tensor scales, the GEMM of the per-tensor dynamic path): sa and sb
+// are single fp32 values, so no per-block promotion is needed -- the MMAs
+// accumulate a unit's whole K range into one TMEM buffer and the epilogue
+// multiplies it by sa*sb once.
 #pragma once
 
 #include <cuda.h>
@@ -56,7 +61,7 @@ struct GemmParams {
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
 struct GemmCfg {
     // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
     // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
@@ -81,7 +86,7 @@ struct GemmCfg {
     static constexpr int kTmemCols = kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
     static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
-    static constexpr int kSlabFloats = SWAP ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
+    static constexpr int kSlabFloats = (SWAP && !PT) ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
                                          + size_t(kSlabFloats) * 4 + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
@@ -142,11 +147,11 @@ __device__ __forceinline__ float pick4(const float4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false>
-__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR>::kThreads, 1)
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
+__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR, PT>::kThreads, 1)
 block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmQ, const GemmParams p) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR>;
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT>;
     constexpr int NB = C::kNumBuf;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -229,44 +234,65 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             // -------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BN, C::kTileRows);
             uint32_t it = 0, c = 0;
-            for (int u = unit0; u < p.units && !*abort_flag; u += unit_step) {
+            bool failed = false;
+            // the most recent commit (a commit arrives once every MMA issued
+            // before it has finished): what an abort must wait for
+            uint64_t* last_bar = nullptr;
+            uint32_t last_parity = 0;
+            for (int u = unit0; u < p.units && !failed; u += unit_step) {
                 int tp, tq, kb0, kb1;
                 unit_coords(p, u, tp, tq, kb0, kb1);
-                for (int kb = kb0; kb < kb1; ++kb, ++it, ++c) {
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
+                // One promotion step = one K block (block scales), or the
+                // whole K range of the unit (per-tensor scales: the MMAs
+                // accumulate every K block into one TMEM buffer).
+                const int steps = PT ? 1 : kb1 - kb0;
+                int kb = kb0;
+                for (int st = 0; st < steps && !failed; ++st, ++c) {
                     const uint32_t buf = c % NB, tph = (c / NB) & 1;
                     const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1, p.wait_budget)
                                             : ptx::mbar_wait(&tempty[buf], tph ^ 1, p.wait_budget);
-                    if (!freed) { fail(); break; }
-                    if (!ptx::mbar_wait(&full[s], ph, p.wait_budget)) { fail(); break; }
-                    ptx::tc_fence_after();
-                    const uint32_t pa = ptx::smem_u32(tiles + size_t(s) * C::kStageBytes);
-                    const uint32_t qa = pa + C::kPBytes;
+                    if (!freed) { fail(); failed = true; break; }
                     const uint32_t d = tmem_base + buf * BN;
-                    if (PAIR) {
+                    const int kb_end = PT ? kb1 : kb + 1;
+                    for (; kb < kb_end; ++kb, ++it) {
+                        const int s = it % STAGES;
+                        const uint32_t ph = (it / STAGES) & 1;
+                        if (!ptx::mbar_wait(&full[s], ph, p.wait_budget)) { fail(); failed = true; break; }
+                        ptx::tc_fence_after();
+                        const uint32_t pa = ptx::smem_u32(tiles + size_t(s) * C::kStageBytes);
+                        const uint32_t qa = pa + C::kPBytes;
+                        const uint32_t first = (PT && kb > kb0) ? 1u : 0u;   // accumulate across K blocks
+                        if (PAIR) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            ptx::mma_f8_pair(d, ptx::sw128_kmajor_desc(pa + 32 * k),
-                                             ptx::sw128_kmajor_desc(qa + 32 * k), idesc, k > 0);
-                        // stage free and partial ready, in both CTAs
-                        const uint32_t e0 = ptx::smem_u32(&empty[s]), f0 = ptx::smem_u32(&tfull[buf]);
-                        ptx::mma_commit_pair(e0);
-                        ptx::mma_commit_pair(ptx::mapa_shared(e0, 1));
+                            for (int k = 0; k < 4; ++k)
+                                ptx::mma_f8_pair(d, ptx::sw128_kmajor_desc(pa + 32 * k),
+                                                 ptx::sw128_kmajor_desc(qa + 32 * k), idesc, first | (k > 0));
+                            const uint32_t e0 = ptx::smem_u32(&empty[s]);      // stage free, in both CTAs
+                            ptx::mma_commit_pair(e0);
+                            ptx::mma_commit_pair(ptx::mapa_shared(e0, 1));
+                        } else {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                ptx::mma_f8(d, ptx::sw128_kmajor_desc(pa + 32 * k),
+                                            ptx::sw128_kmajor_desc(qa + 32 * k), idesc, first | (k > 0));
+                            ptx::mma_commit(&empty[s]);
+                        }
+                        last_bar = &empty[s];
+                        last_parity = ph;
+                    }
+                    if (failed) break;
+                    if (PAIR) {                                              // step ready, in both CTAs
+                        const uint32_t f0 = ptx::smem_u32(&tfull[buf]);
                         ptx::mma_commit_pair(f0);
                         ptx::mma_commit_pair(ptx::mapa_shared(f0, 1));
                     } else {
-#pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            ptx::mma_f8(d, ptx::sw128_kmajor_desc(pa + 32 * k),
-                                        ptx::sw128_kmajor_desc(qa + 32 * k), idesc, k > 0);
-                        ptx::mma_commit(&empty[s]);
                         ptx::mma_commit(&tfull[buf]);
                     }
+                    last_bar = &tfull[buf];
+                    last_parity = tph;
                 }
             }
-            if (*abort_flag && c > 0)
-                ptx::mbar_wait(&tfull[(c - 1) % NB], ((c - 1) / NB) & 1, 100000000LL);
+            if (*abort_flag && last_bar) ptx::mbar_wait(last_bar, last_parity, 100000000LL);
         }
         __syncwarp();
     } else {
@@ -290,7 +316,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             const int q0 = tq * BN;
             const int m_row = tp * C::kTileRows + int(rank) * 128 + row;   // normal: token row
             const int n_row = tp * 128 + row;                              // swapped: weight row
-            if (SWAP) {
+            if (SWAP && !PT) {
                 // slab[kbl*BN + j] = sa[q0+j, kb0+kbl] * sb[tp, kb0+kbl]
                 ptx::named_bar_sync(1, nthreads);
                 for (int i = etid; i < nkb * BN; i += nthreads) {
@@ -309,21 +335,24 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             // Normal mode: row scale sa[m_row, kb] times the column block's
             // sb[nb, kb], fetched four K blocks at a time, one group ahead.
             const int nb = (q0 + chalf * C::kCW) >> 7;
-            const bool row_ok = !SWAP && m_row < p.M;
-            const bool col_ok = !SWAP && nb * 128 < p.N;
+            const bool row_ok = !SWAP && !PT && m_row < p.M;
+            const bool col_ok = !SWAP && !PT && nb * 128 < p.N;
             const float* sa_row = p.sa + int64_t(SWAP ? 0 : (row_ok ? m_row : 0)) * p.G;
             const float* sb_row = p.sb + int64_t(col_ok ? nb : 0) * p.G;
             float4 sa_cur, sb_cur, sa_nxt, sb_nxt;
-            if (!SWAP) {
+            if (!SWAP && !PT) {
                 sa_cur = load_scale4(sa_row, kb0 >> 2, p.G, vec4, row_ok);
                 sb_cur = load_scale4(sb_row, kb0 >> 2, p.G, vec4, col_ok);
                 sa_nxt = load_scale4(sa_row, (kb0 >> 2) + 1, p.G, vec4, row_ok);
                 sb_nxt = load_scale4(sb_row, (kb0 >> 2) + 1, p.G, vec4, col_ok);
             }
             bool ok = true;
-            for (int kb = kb0; kb < kb1; ++kb, ++c) {
-                float s = 0.0f;
-                if (!SWAP) {
+            // per-tensor scales: one step per unit, one scalar scale
+            const int kb_last = PT ? kb0 + 1 : kb1;
+            const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : 0.0f;
+            for (int kb = kb0; kb < kb_last; ++kb, ++c) {
+                float s = s_pt;
+                if (!SWAP && !PT) {
                     if ((kb & 3) == 0 && kb != kb0) {
                         sa_cur = sa_nxt;
                         sb_cur = sb_nxt;
@@ -359,7 +388,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                             else ptx::mbar_arrive(&tempty[buf]);
                         }
                     }
-                    if (SWAP) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
+                    if (SWAP && !PT) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
                     else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
                 }
             }

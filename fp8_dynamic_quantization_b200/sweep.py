@@ -122,9 +122,25 @@ def run_gemm(t, dev, m, n, k, reps, modes, hbm, fp8):
               "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
 
 
+def run_gemm_pt(t, dev, m, n, k, reps, modes, hbm, fp8):
+    qa, _, qb, _ = inputs.gemm_operands(m, n, k)
+    tqa = torch.from_numpy(qa).to(dev).view(torch.float8_e4m3fn)
+    tqb = torch.from_numpy(qb).to(dev).view(torch.float8_e4m3fn)
+    sa = torch.tensor([0.01], device=dev)
+    sb = torch.tensor([0.02], device=dev)
+    y = torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
+    nbytes = m * k + n * k + 8.0 + 2.0 * m * n
+    flops = 2.0 * m * n * k
+    for mode in modes:
+        us = getattr(t, mode)(lambda: fq.gemm_per_tensor(tqa, sa, tqb, sb, out=y), reps)
+        emit({"op": "gemm_per_tensor", "M": m, "N": n, "K": k, "mode": mode, "us": us,
+              "TFLOP/s": flops / us / 1e6, "frac_fp8": flops / us / 1e6 / fp8,
+              "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm"], default="all")
+    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt"], default="all")
     ap.add_argument("--m", type=int)
     ap.add_argument("--n", type=int)
     ap.add_argument("--k", type=int)
@@ -142,6 +158,8 @@ def main():
         run_group(t, dev, a.m, a.k or 7168, a.reps, modes, hbm)
     elif a.op == "gemm":
         run_gemm(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
+    elif a.op == "gemm_pt":
+        run_gemm_pt(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     else:
         emit({"peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src}})
         for m, _, k in inputs.WORKLOAD_SHAPES[2]:
@@ -151,6 +169,8 @@ def main():
         run_group(t, dev, 64, 2048, a.reps, modes, hbm)
         for m, n, k in inputs.WORKLOAD_SHAPES[1] + inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
             run_gemm(t, dev, m, n, k, a.reps, modes, hbm, fp8)
+        for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
+            run_gemm_pt(t, dev, m, n, k, a.reps, modes, hbm, fp8)
     if fq.device_status() != 0:
         raise SystemExit("device-side error recorded")
 

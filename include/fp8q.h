@@ -174,6 +174,25 @@ int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Per-tensor-scaled FP8 GEMM ([P2] Description and walkthrough: the   */
+/* linear method's dynamic path quantises the input per tensor, then    */
+/* runs the projection GEMM on the codes with the tensor scales)         */
+/* ------------------------------------------------------------------ */
+
+/* Y = bf16_rne( sa * sb * sum_k A[m,k] * B[n,k] ), fp32 accumulation.
+ *   qa: E4M3 [M,K] (row stride lda), sa: ONE fp32 on the device (A's scale)
+ *   qb: E4M3 [N,K] (row stride ldb), sb: ONE fp32 on the device (B's scale)
+ *   y : bf16 [M,N] (row stride ldy)
+ * Shapes, alignment, launch selection and errors as fp8_block_gemm; the
+ * workspace size is fp8_block_gemm_workspace_size(M, N, K).  With scalar
+ * scales there is no per-block promotion: the tensor cores accumulate the
+ * whole K range in TMEM and the epilogue multiplies by sa*sb once. */
+int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa,
+                        const uint8_t* qb, int64_t ldb, const float* sb,
+                        void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Block-scaled FP8 GEMM without any allocation                         */
 /* ------------------------------------------------------------------ */
 

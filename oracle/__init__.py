@@ -221,6 +221,18 @@ def block_gemm_points(qa, sa, qb, sb, ms, ns):
     return R, T
 
 
+def gemm_per_tensor(qa, s_a, qb, s_b):
+    """(R, T) of the per-tensor-scaled GEMM Y = s_a * s_b * A * B^T ([P2]
+    Description and walkthrough: the input is quantised per tensor and the
+    projection runs on the codes with the tensor scales): the block GEMM's
+    definition with every block scale equal to the tensor scale."""
+    m, k = qa.shape
+    n = qb.shape[0]
+    sa = np.full((m, k // 128), np.float32(s_a), dtype=np.float32)
+    sb = np.full(((n + 127) // 128, k // 128), np.float32(s_b), dtype=np.float32)
+    return block_gemm(qa, sa, qb, sb)
+
+
 def f64_to_bf16(values) -> np.ndarray:
     """bf16 bit patterns (uint16) of float64 values, round-to-nearest-even."""
     v = np.ascontiguousarray(np.asarray(values, dtype=np.float64))

@@ -26,15 +26,23 @@ for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 25
     Y = y.float().cpu().numpy().astype(np.float64)
     bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
     assert bad == 0, (m, n, k, bad)
+    # per-tensor scales; a forced pair row runs it as the single-CTA tile
+    s_a, s_b = np.float32(0.05), np.float32(0.003)
+    y = fq.gemm_per_tensor(torch.from_numpy(qa).to(dev), torch.tensor([s_a], device=dev),
+                           torch.from_numpy(qb).to(dev), torch.tensor([s_b], device=dev))
+    R, T = oracle.gemm_per_tensor(qa, s_a, qb, s_b)
+    Y = y.float().cpu().numpy().astype(np.float64)
+    bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
+    assert bad == 0, ("per-tensor", m, n, k, bad)
 assert fq.device_status() == 0
 print("ok")
 '''
 
 
 @pytest.mark.parametrize("tile", ["normal:128", "normal:192", "normal:256", "pair:256", "pair:128",
-                                  "swap:16", "swap:64", "swap:128:3"])
+                                  "swap:16", "swap:32", "swap:64", "swap:128:3"])
 def test_gemm_mode_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
     env = dict(os.environ, FP8Q_GEMM_TILE=tile)
-    r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True,
+    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, tile], env=env, capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr

@@ -415,3 +415,15 @@ def test_quant_apply_matches_per_tensor(oracle_mod):
     q3, s3 = oracle_mod.quant_apply(bits, 0)
     assert s3 == 0
     np.testing.assert_array_equal(q3, np.where(np.signbit(x.float().numpy()), 0x80, 0).astype(np.uint8))
+
+
+def test_gemm_per_tensor_is_scaled_integer_matmul(oracle_mod):
+    """Per-tensor scales: R = s_a * s_b * (A_dec @ B_dec^T), the inner sum exact."""
+    qa, _, qb, _ = inputs.gemm_operands(7, 260, 512, seed=21)
+    s_a, s_b = np.float32(0.0371), np.float32(0.00917)
+    R, T = oracle_mod.gemm_per_tensor(qa, s_a, qb, s_b)
+    A = torch.from_numpy(torch_decode(qa))
+    B = torch.from_numpy(torch_decode(qb))
+    ref = (float(s_a) * float(s_b)) * (A @ B.T).numpy()
+    np.testing.assert_allclose(R, ref, rtol=1e-12)
+    np.testing.assert_allclose(T, (float(s_a) * float(s_b)) * (A.abs() @ B.abs().T).numpy(), rtol=1e-12)
