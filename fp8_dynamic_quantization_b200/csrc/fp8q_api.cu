@@ -52,11 +52,11 @@ constexpr int kStreamU = 4;         // vectors per thread per iteration elsewher
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
 cudaError_t set_gemm_smem() {
-    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT>,
+    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT, SS>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(GemmCfg<BN, SWAP, STAGES, PAIR, PT>::kSmemBytes));
+                                int(GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>::kSmemBytes));
 }
 
 // Device facts, queried once per device.  FP8Q_ERR_NO_DEVICE unless the
@@ -88,6 +88,8 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, true>();
@@ -274,12 +276,29 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
-void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams& p, int grid,
-                 cudaStream_t st) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT>;
+// Map of an fp32 scale matrix [rows, G] (row pitch G floats, G % 4 == 0,
+// 16-byte aligned base): boxes of 4 consecutive K-block scales x box_rows
+// rows, no swizzle; rows past the end read as zero.
+bool make_scale_tmap(CUtensorMap* m, const float* base, int64_t rows, int64_t G, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(G), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(G) * 4};
+    cuuint32_t box[2] = {4u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// tsa/tsb: scale maps (staged-scale variants only; the others ignore them)
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
+void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& tsa, const CUtensorMap& tsb,
+                 const GemmParams& p, int grid, cudaStream_t st) {
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>;
     if (!PAIR) {
-        block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT><<<grid, C::kThreads, C::kSmemBytes, st>>>(tp, tq, p);
+        block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT, SS><<<grid, C::kThreads, C::kSmemBytes, st>>>(
+            tp, tq, tsa, tsb, p);
         return;
     }
     cudaLaunchConfig_t cfg = {};
@@ -294,7 +313,7 @@ void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const GemmParams&
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR>, tp, tq, p);
+    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR>, tp, tq, tsa, tsb, p);
 }
 
 // ------------------------------------------------------------------ no-alloc GEMM scratch
@@ -585,41 +604,50 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     p.splits = pl.splits;
     p.units = pl.units;
     p.scale_vec4 = !per_tensor && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
+    // Normal 128/256-wide tiles stage the block scales through shared memory
+    // (TMA boxes of 4 K blocks) when the scale rows allow 16-byte boxes.
+    const bool staged = p.scale_vec4 && !pl.swap && !pl.pair && (pl.bn == 128 || pl.bn == 256);
+    CUtensorMap tsa = tp, tsb = tq;
+    if (staged && (!make_scale_tmap(&tsa, sa, M, p.G, 128) ||
+                   !make_scale_tmap(&tsb, sb, (N + 127) / 128, p.G, pl.bn / 128)))
+        return FP8Q_ERR_CUDA;
     p.wait_budget = wait_budget_cycles();
     if (log_enabled())
-        std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s bn=%d stages=%d splits=%d units=%d grid=%d\n",
+        std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d\n",
                      (long long)M, (long long)N, (long long)K,
-                     pl.swap ? "swap" : pl.pair ? "pair" : "normal", pl.bn,
+                     pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
     if (per_tensor) {
         if (pl.swap) {
             switch (pl.bn) {
-                case 16: launch_gemm<16, true, 12, false, true>(tp, tq, p, pl.grid, st); break;
-                case 32: launch_gemm<32, true, 10, false, true>(tp, tq, p, pl.grid, st); break;
-                case 64: launch_gemm<64, true, 8, false, true>(tp, tq, p, pl.grid, st); break;
-                default: launch_gemm<128, true, 6, false, true>(tp, tq, p, pl.grid, st); break;
+                case 16: launch_gemm<16, true, 12, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 32: launch_gemm<32, true, 10, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 64: launch_gemm<64, true, 8, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                default: launch_gemm<128, true, 6, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
             }
         } else if (pl.bn == 128) {
-            launch_gemm<128, false, 6, false, true>(tp, tq, p, pl.grid, st);
+            launch_gemm<128, false, 6, false, true>(tp, tq, tsa, tsb, p, pl.grid, st);
         } else if (pl.bn == 192) {
-            launch_gemm<192, false, 5, false, true>(tp, tq, p, pl.grid, st);
+            launch_gemm<192, false, 5, false, true>(tp, tq, tsa, tsb, p, pl.grid, st);
         } else {
-            launch_gemm<256, false, 4, false, true>(tp, tq, p, pl.grid, st);
+            launch_gemm<256, false, 4, false, true>(tp, tq, tsa, tsb, p, pl.grid, st);
         }
     } else if (pl.swap) {
         switch (pl.bn) {
-            case 16: launch_gemm<16, true, 12>(tp, tq, p, pl.grid, st); break;
-            case 32: launch_gemm<32, true, 10>(tp, tq, p, pl.grid, st); break;
-            case 64: launch_gemm<64, true, 8>(tp, tq, p, pl.grid, st); break;
-            default: launch_gemm<128, true, 6>(tp, tq, p, pl.grid, st); break;
+            case 16: launch_gemm<16, true, 12>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+            case 32: launch_gemm<32, true, 10>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+            case 64: launch_gemm<64, true, 8>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+            default: launch_gemm<128, true, 6>(tp, tq, tsa, tsb, p, pl.grid, st); break;
         }
     } else if (pl.pair) {
-        if (pl.bn == 256) launch_gemm<256, false, 6, true>(tp, tq, p, pl.grid, st);
-        else launch_gemm<128, false, 8, true>(tp, tq, p, pl.grid, st);
+        if (pl.bn == 256) launch_gemm<256, false, 6, true>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else launch_gemm<128, false, 8, true>(tp, tq, tsa, tsb, p, pl.grid, st);
     } else {
-        if (pl.bn == 192) launch_gemm<192, false, 5>(tp, tq, p, pl.grid, st);
-        else if (pl.bn == 256) launch_gemm<256, false, 4>(tp, tq, p, pl.grid, st);
-        else launch_gemm<128, false, 6>(tp, tq, p, pl.grid, st);
+        if (pl.bn == 192) launch_gemm<192, false, 5>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else if (pl.bn == 256 && staged) launch_gemm<256, false, 4, false, false, true>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else if (pl.bn == 256) launch_gemm<256, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else if (staged) launch_gemm<128, false, 6, false, false, true>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else launch_gemm<128, false, 6>(tp, tq, tsa, tsb, p, pl.grid, st);
     }
     if ((rc = launch_status()) != FP8Q_OK) return rc;
     if (pl.splits > 1) {

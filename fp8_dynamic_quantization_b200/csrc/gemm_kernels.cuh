@@ -61,7 +61,7 @@ struct GemmParams {
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
 struct GemmCfg {
     // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
     // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
@@ -87,8 +87,15 @@ struct GemmCfg {
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
     static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
     static constexpr int kSlabFloats = (SWAP && !PT) ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
+    // SS: block scales staged through shared memory.  The producer copies,
+    // per group of 4 K blocks, the tile's 128 x 4 row scales and its
+    // BN/128 x 4 column-block scales into a ring of kScaleSlots slots.
+    static constexpr int kScaleSlots = SS ? 4 : 0;
+    static constexpr int kSbRows = BN / 128;                   // column blocks per tile (SS)
+    static constexpr int kScaleSlotBytes = 2048 + 128;         // 128 x 4 fp32, then kSbRows x 4 fp32
+    static constexpr uint32_t kScaleTx = 2048 + 16 * kSbRows;  // bytes one slot receives
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
-                                         + size_t(kSlabFloats) * 4 + 512;
+                                         + size_t(kSlabFloats) * 4 + size_t(kScaleSlots) * kScaleSlotBytes + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(kCW % 16 == 0, "columns per thread");
     static_assert(!SWAP || BN <= 128, "swapped tiles hold at most 128 tokens");
@@ -98,7 +105,8 @@ struct GemmCfg {
     static_assert(!PAIR || (!SWAP && (BN == 256 || BN == 128)), "CTA pairs compute 256 x 256 or 256 x 128 tiles");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kSmemBytes <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * kNumBuf) * 8 + 8 <= 512, "barrier area");
+    static_assert((2 * STAGES + 2 * kNumBuf + 2 * kScaleSlots) * 8 + 8 <= 512, "barrier area");
+    static_assert(!SS || (!SWAP && !PAIR && !PT && (BN == 128 || BN == 256)), "staged scales: normal 128/256 tiles");
 };
 
 __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp, int& tq,
@@ -147,24 +155,30 @@ __device__ __forceinline__ float pick4(const float4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false>
-__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR, PT>::kThreads, 1)
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
+__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>::kThreads, 1)
 block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
-                  const __grid_constant__ CUtensorMap tmQ, const GemmParams p) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT>;
+                  const __grid_constant__ CUtensorMap tmQ,
+                  const __grid_constant__ CUtensorMap tmSA,    // row scales [M, G] fp32 (SS only)
+                  const __grid_constant__ CUtensorMap tmSB,    // column-block scales [NB, G] fp32 (SS only)
+                  const GemmParams p) {
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>;
     constexpr int NB = C::kNumBuf;
+    constexpr uint32_t kSlots = C::kScaleSlots > 0 ? C::kScaleSlots : 1;   // divisor for the (SS) slot ring
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* tiles = smem;                                        // STAGES x (P | Q)
     float* slab = reinterpret_cast<float*>(smem + size_t(STAGES) * C::kStageBytes);
-    uint64_t* bars = reinterpret_cast<uint64_t*>(
-        smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4);
+    uint8_t* sring = smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4;   // SS slots
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sring + size_t(C::kScaleSlots) * C::kScaleSlotBytes);
     uint64_t* full = bars;                        // [STAGES] TMA landed
     uint64_t* empty = bars + STAGES;              // [STAGES] MMA done reading
     uint64_t* tfull = bars + 2 * STAGES;          // [NB] block partial ready in TMEM
     uint64_t* tempty = bars + 2 * STAGES + NB;    // [NB] promotion done reading TMEM
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 2 * NB);
+    uint64_t* sfull = bars + 2 * STAGES + 2 * NB;  // [kScaleSlots] scale slot landed (SS)
+    uint64_t* sempty = sfull + C::kScaleSlots;     // [kScaleSlots] scale slot read by every promotion warp
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(sempty + C::kScaleSlots);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -180,10 +194,18 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             ptx::mbar_init(&tfull[b], 1);
             ptx::mbar_init(&tempty[b], (PAIR ? 2 : 1) * 4 * C::kEpiWG);
         }
+        for (int i = 0; i < C::kScaleSlots; ++i) {
+            ptx::mbar_init(&sfull[i], 1);
+            ptx::mbar_init(&sempty[i], 4 * C::kEpiWG);
+        }
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
-    if (warp == 0 && lane == 0) { ptx::prefetch_tmap(&tmP); ptx::prefetch_tmap(&tmQ); }
+    if (warp == 0 && lane == 0) {
+        ptx::prefetch_tmap(&tmP);
+        ptx::prefetch_tmap(&tmQ);
+        if (SS) { ptx::prefetch_tmap(&tmSA); ptx::prefetch_tmap(&tmSB); }
+    }
     if (warp == 1) {
         if (PAIR) { ptx::tmem_alloc_pair(tmem_base_smem, C::kTmemCols); ptx::tmem_relinquish_pair(); }
         else { ptx::tmem_alloc(tmem_base_smem, C::kTmemCols); ptx::tmem_relinquish(); }
@@ -201,15 +223,27 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- producer
             uint32_t it = 0;
-            for (int u = unit0; u < p.units && !*abort_flag; u += unit_step) {
+            uint32_t sg = 0;             // scale groups issued (SS)
+            bool stop = false;
+            for (int u = unit0; u < p.units && !*abort_flag && !stop; u += unit_step) {
                 int tp, tq, kb0, kb1;
                 unit_coords(p, u, tp, tq, kb0, kb1);
                 const int prow = tp * C::kTileRows + int(rank) * 128;
                 const int qrow = tq * BN + int(rank) * C::kQRows;
                 for (int kb = kb0; kb < kb1; ++kb, ++it) {
+                    if (SS && (kb == kb0 || (kb & 3) == 0)) {
+                        // scales of K blocks [4*(kb/4), 4*(kb/4)+4): x is a multiple of 4 fp32
+                        const uint32_t slot = sg % kSlots, sph = (sg / kSlots) & 1;
+                        if (!ptx::mbar_wait(&sempty[slot], sph ^ 1, p.wait_budget)) { fail(); stop = true; break; }
+                        uint8_t* sdst = sring + size_t(slot) * C::kScaleSlotBytes;
+                        ptx::mbar_arrive_expect_tx(&sfull[slot], C::kScaleTx);
+                        ptx::tma_load_2d(sdst, &tmSA, &sfull[slot], (kb >> 2) * 4, prow);
+                        ptx::tma_load_2d(sdst + 2048, &tmSB, &sfull[slot], (kb >> 2) * 4, tq * C::kSbRows);
+                        ++sg;
+                    }
                     const int s = it % STAGES;
                     const uint32_t ph = (it / STAGES) & 1;
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, p.wait_budget)) { fail(); break; }
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, p.wait_budget)) { fail(); stop = true; break; }
                     uint8_t* dst = tiles + size_t(s) * C::kStageBytes;
                     if (PAIR) {
                         // both CTAs' copies complete on the leader's barrier
@@ -229,6 +263,9 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 const uint32_t first = it > STAGES ? it - STAGES : 0;
                 for (uint32_t j = first; j < it; ++j)
                     ptx::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 100000000LL);
+                const uint32_t sfirst = sg > uint32_t(C::kScaleSlots) ? sg - C::kScaleSlots : 0;
+                for (uint32_t g = sfirst; g < sg; ++g)
+                    ptx::mbar_wait(&sfull[g % kSlots], (g / kSlots) & 1, 100000000LL);
             }
         } else if (warp == 1 && lane == 0 && leader) {
             // -------------------------------------------------------- MMA issuer
@@ -306,6 +343,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         const int etid = threadIdx.x - 128;
         const bool vec4 = p.scale_vec4 != 0;
         uint32_t c = 0;
+        uint32_t sg = 0;                          // scale groups consumed (SS)
         uint64_t acc2[C::kCW / 2];
         // the leader's tempty barriers, as cluster addresses (pair mode)
         const uint32_t tempty0 = PAIR ? ptx::mapa_shared(ptx::smem_u32(tempty), 0) : 0u;
@@ -340,7 +378,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             const float* sa_row = p.sa + int64_t(SWAP ? 0 : (row_ok ? m_row : 0)) * p.G;
             const float* sb_row = p.sb + int64_t(col_ok ? nb : 0) * p.G;
             float4 sa_cur, sb_cur, sa_nxt, sb_nxt;
-            if (!SWAP && !PT) {
+            if (!SWAP && !PT && !SS) {
                 sa_cur = load_scale4(sa_row, kb0 >> 2, p.G, vec4, row_ok);
                 sb_cur = load_scale4(sb_row, kb0 >> 2, p.G, vec4, col_ok);
                 sa_nxt = load_scale4(sa_row, (kb0 >> 2) + 1, p.G, vec4, row_ok);
@@ -352,7 +390,21 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : 0.0f;
             for (int kb = kb0; kb < kb_last; ++kb, ++c) {
                 float s = s_pt;
-                if (!SWAP && !PT) {
+                if (SS) {
+                    if (kb == kb0 || (kb & 3) == 0) {
+                        // this group's scales: row `row` of the 128 x 4 box, and
+                        // the column block of this thread's slice
+                        const uint32_t slot = sg % kSlots, sph = (sg / kSlots) & 1;
+                        if (!ptx::mbar_wait(&sfull[slot], sph, p.wait_budget)) { fail(); ok = false; break; }
+                        const uint8_t* src = sring + size_t(slot) * C::kScaleSlotBytes;
+                        sa_cur = *reinterpret_cast<const float4*>(src + row * 16);
+                        sb_cur = *reinterpret_cast<const float4*>(src + 2048 + ((chalf * C::kCW) >> 7) * 16);
+                        __syncwarp();
+                        if (lane == 0) ptx::mbar_arrive(&sempty[slot]);
+                        ++sg;
+                    }
+                    s = pick4(sa_cur, kb & 3) * pick4(sb_cur, kb & 3);
+                } else if (!SWAP && !PT) {
                     if ((kb & 3) == 0 && kb != kb0) {
                         sa_cur = sa_nxt;
                         sb_cur = sb_nxt;

@@ -62,6 +62,9 @@ def sample_points(M, N, g, n_random=4096):
     (1, 8, 128), (1, 128, 128), (3, 200, 256), (16, 300, 1024), (17, 520, 384),
     (40, 2048, 2048), (64, 2048, 2048), (100, 256, 7168), (128, 384, 512),
     (130, 300, 512), (256, 384, 1024), (600, 520, 384), (700, 1000, 1280), (1025, 264, 256),
+    # scale rows in 16-byte boxes (K/128 % 4 == 0): ragged M, N past the last
+    # weight block, split-K ranges starting inside a group of 4 K blocks
+    (300, 600, 2048), (520, 300, 512), (520, 640, 1536), (200, 1100, 3072),
 ])
 def test_gemm_small_full(oracle_mod, gpu, m, n, k):
     qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m * 131 + n * 7 + k)
