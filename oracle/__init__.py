@@ -71,6 +71,10 @@ def _load():
         lib.oracle_quant_apply.argtypes = [_p, _i64, _i64, _i64, ctypes.c_uint16, _p, _i64, _p]
         lib.oracle_quant_group128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_quant_block128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
+        lib.oracle_e8m0_from_amax.argtypes = [ctypes.c_float]
+        lib.oracle_e8m0_from_amax.restype = ctypes.c_int
+        lib.oracle_quant_group128_ue8m0.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
+        lib.oracle_quant_block128_ue8m0.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_block_gemm.argtypes = [_p, _i64, _p, _p, _i64, _p,
                                           _i64, _i64, _i64, _p, _p]
         lib.oracle_block_gemm_points.argtypes = [_p, _i64, _p, _p, _i64, _p,
@@ -182,6 +186,45 @@ def quant_block128(w_bits: np.ndarray):
     return q, s
 
 
+# ---------------------------------------------------------------- ue8m0
+# [P1] "Benchmarking the Activation Quantization Kernel" names the ue8m0
+# scale format (scale_fmt="ue8m0"); the reading of it (smallest power of two
+# >= amax/448, E8M0 byte = exponent + 127, 255 = NaN) is in fp8q_oracle.c.
+def e8m0_from_amax(amax: float) -> int:
+    """E8M0 byte of the power-of-two scale for a group amax."""
+    return int(_load().oracle_e8m0_from_amax(float(amax)))
+
+
+def e8m0_to_f32(b) -> np.ndarray:
+    """fp32 values 2^(b-127) of E8M0 bytes (NaN for 255)."""
+    b = np.asarray(b, dtype=np.uint8)
+    out = np.ldexp(np.ones(b.shape, dtype=np.float64), b.astype(np.int64) - 127).astype(np.float32)
+    out[b == 255] = np.nan
+    return out
+
+
+def quant_group128_ue8m0(x_bits: np.ndarray):
+    """(codes [M,K] uint8, E8M0 scale bytes [M,K/128] uint8)."""
+    m, k, ld = _rows(x_bits, 2)
+    if k % 128:
+        raise ValueError("K must be a multiple of 128")
+    q = np.empty((m, k), dtype=np.uint8)
+    s = np.empty((m, k // 128), dtype=np.uint8)
+    _load().oracle_quant_group128_ue8m0(_ptr(x_bits), m, k, ld, _ptr(q), k, _ptr(s))
+    return q, s
+
+
+def quant_block128_ue8m0(w_bits: np.ndarray):
+    """(codes [N,K] uint8, E8M0 scale bytes [ceil(N/128),K/128] uint8)."""
+    n, k, ld = _rows(w_bits, 2)
+    if k % 128:
+        raise ValueError("K must be a multiple of 128")
+    q = np.empty((n, k), dtype=np.uint8)
+    s = np.empty(((n + 127) // 128, k // 128), dtype=np.uint8)
+    _load().oracle_quant_block128_ue8m0(_ptr(w_bits), n, k, ld, _ptr(q), k, _ptr(s))
+    return q, s
+
+
 # ---------------------------------------------------------------- GEMM
 def _gemm_args(qa, sa, qb, sb):
     m, k, lda = _rows(qa, 1)
@@ -231,6 +274,17 @@ def gemm_per_tensor(qa, s_a, qb, s_b):
     sa = np.full((m, k // 128), np.float32(s_a), dtype=np.float32)
     sb = np.full(((n + 127) // 128, k // 128), np.float32(s_b), dtype=np.float32)
     return block_gemm(qa, sa, qb, sb)
+
+
+def gemm_ue8m0(qa, sa_bytes, qb, sb_bytes):
+    """(R, T) of the block GEMM with E8M0 scale bytes: the block GEMM's
+    definition with each scale 2^(b-127)."""
+    return block_gemm(qa, e8m0_to_f32(sa_bytes), qb, e8m0_to_f32(sb_bytes))
+
+
+def gemm_ue8m0_points(qa, sa_bytes, qb, sb_bytes, ms, ns):
+    """gemm_ue8m0 at the listed (m, n) points."""
+    return block_gemm_points(qa, e8m0_to_f32(sa_bytes), qb, e8m0_to_f32(sb_bytes), ms, ns)
 
 
 def f64_to_bf16(values) -> np.ndarray:

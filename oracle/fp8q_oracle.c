@@ -28,6 +28,13 @@
  * definition; an all-zero tensor or group gets scale 0 and signed-zero codes;
  * NaN propagates through amax; NaN codes are 0x7F (sign not significant).
  *
+ * The ue8m0 variant ([P1] "Benchmarking the Activation Quantization Kernel"
+ * passes scale_fmt="ue8m0" and says nothing more): the scale is a power of two
+ * stored as an E8M0 byte b (value 2^(b-127), b = 255 is NaN), namely the
+ * smallest 2^e >= amax/448, with e clamped to [-127, 127]; an all-zero group
+ * gets b = 0; an Inf or NaN amax gives b = 255 and NaN codes (0x7F).  Codes
+ * are e4m3_rne(x * 2^-e), exact before the one rounding.
+ *
  * Everything below is loops over elements.  No SIMD intrinsics, no blocking,
  * no reordering beyond what the definitions say.  OpenMP only splits
  * independent rows / groups across threads.
@@ -286,6 +293,61 @@ void oracle_quant_block128(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
             for (int64_t r = r0; r < r1; r++)
                 for (int64_t c = 128 * g; c < 128 * g + 128; c++)
                     q[r * ldq + c] = quant_one(w[r * ldw + c], s);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
+/* ue8m0 (power-of-two) scales ([P1] "Benchmarking the Activation        */
+/* Quantization Kernel": act_quant(..., scale_fmt="ue8m0")).  The pages  */
+/* name the format only; the reading is in the header comment above.    */
+/* ------------------------------------------------------------------ */
+
+/* E8M0 byte of the scale for a group amax: the smallest e in
+   [-127, 127] with 448 * 2^e >= amax, plus the bias 127; 255 for Inf/NaN. */
+int oracle_e8m0_from_amax(float amax) {
+    if (isnan(amax) || isinf(amax)) return 255;
+    double a = (double)amax;
+    int e = -127;
+    while (e < 127 && ldexp(448.0, e) < a) e++;
+    return e + 127;
+}
+
+/* One element's code for an E8M0 scale byte: NaN (0x7F) for byte 255,
+   else e4m3_rne(x * 2^-(b-127)) -- the product is exact in double. */
+static uint8_t quant_one_e8m0(uint16_t xb, int b) {
+    if (b == 255) return 0x7F;
+    double v = (double)bf16_bits_to_f32(xb) * ldexp(1.0, 127 - b);
+    return oracle_e4m3_encode((float)v);   /* |v| <= 448: exact in fp32 unless below 2^-126 */
+}
+
+void oracle_quant_group128_ue8m0(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                 uint8_t* q, int64_t ldq, uint8_t* sbytes) {
+    int64_t G = K / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; r++) {
+        for (int64_t g = 0; g < G; g++) {
+            int b = oracle_e8m0_from_amax(amax_bf16(x, ldx, r, r + 1, 128 * g, 128 * g + 128));
+            sbytes[r * G + g] = (uint8_t)b;
+            for (int64_t c = 128 * g; c < 128 * g + 128; c++)
+                q[r * ldq + c] = quant_one_e8m0(x[r * ldx + c], b);
+        }
+    }
+}
+
+void oracle_quant_block128_ue8m0(const uint16_t* w, int64_t N, int64_t K, int64_t ldw,
+                                 uint8_t* q, int64_t ldq, uint8_t* sbytes) {
+    int64_t G = K / 128;
+    int64_t NB = (N + 127) / 128;
+    #pragma omp parallel for schedule(static)
+    for (int64_t nb = 0; nb < NB; nb++) {
+        int64_t r0 = nb * 128, r1 = (nb * 128 + 128 < N) ? nb * 128 + 128 : N;
+        for (int64_t g = 0; g < G; g++) {
+            int b = oracle_e8m0_from_amax(amax_bf16(w, ldw, r0, r1, 128 * g, 128 * g + 128));
+            sbytes[nb * G + g] = (uint8_t)b;
+            for (int64_t r = r0; r < r1; r++)
+                for (int64_t c = 128 * g; c < 128 * g + 128; c++)
+                    q[r * ldq + c] = quant_one_e8m0(w[r * ldw + c], b);
         }
     }
 }

@@ -427,3 +427,117 @@ def test_gemm_per_tensor_is_scaled_integer_matmul(oracle_mod):
     ref = (float(s_a) * float(s_b)) * (A @ B.T).numpy()
     np.testing.assert_allclose(R, ref, rtol=1e-12)
     np.testing.assert_allclose(T, (float(s_a) * float(s_b)) * (A.abs() @ B.abs().T).numpy(), rtol=1e-12)
+
+
+# ---------------------------------------------------------------- ue8m0
+# The ue8m0 reading: scale = smallest power of two 2^e >= amax/448, e clamped
+# to [-127, 127], stored as the E8M0 byte e + 127 (255 = NaN).
+
+def _bf16_groups(rows):
+    """bf16 bit patterns [len(rows), 128] from float rows (exactly representable)."""
+    t = torch.tensor(np.asarray(rows, dtype=np.float32)).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def test_e8m0_exponent_matches_log2(oracle_mod):
+    """Every finite bf16 magnitude: byte = clamp(ceil(log2(a/448))) + 127, by the
+    math library's log2 (a/448 is never within 1/224 of a power of two from
+    above, so float64 log2 decides the ceiling exactly)."""
+    bits = np.arange(1, 0x7F80, dtype=np.uint32)
+    a = (bits << 16).view(np.float32).astype(np.float64)
+    want = np.clip(np.ceil(np.log2(a / 448.0)), -127, 127).astype(np.int64) + 127
+    got = np.array([oracle_mod.e8m0_from_amax(float(v)) for v in a])
+    assert np.array_equal(got, want)
+    assert oracle_mod.e8m0_from_amax(0.0) == 0
+    assert oracle_mod.e8m0_from_amax(float("inf")) == 255
+    assert oracle_mod.e8m0_from_amax(float("nan")) == 255
+
+
+def test_ue8m0_worked_values(oracle_mod):
+    x = _bf16_groups([[1.0] * 128, [448.0] + [3.0] * 127, [450.0] + [-1.0] * 127])
+    q, s = oracle_mod.quant_group128_ue8m0(x)
+    assert s[:, 0].tolist() == [119, 127, 128]            # 2^-8, 2^0, 2^1
+    dec = oracle_mod.e4m3_decode
+    assert set(dec(q[0]).tolist()) == {256.0}               # 1.0 * 2^8
+    assert dec(q[1, 0]) == 448.0 and dec(q[1, 1]) == 3.0
+    assert dec(q[2, 0]) == 224.0                            # 450/2 = 225 -> 224 (RNE, spacing 16)
+    assert dec(q[2, 1]) == -0.5
+
+
+def test_ue8m0_agrees_with_fp32_path_on_power_of_two_ratios(oracle_mod):
+    """When amax/448 is a power of two the fp32 scale is that power of two, so
+    both readings give the same codes and the same scale value."""
+    g = np.random.default_rng(3)
+    rows = []
+    for k in range(-20, 21, 5):
+        r = g.normal(0, 1, 128) * 448.0 * 2.0 ** k / 6.0
+        r = np.clip(r, -0.99 * 448 * 2.0 ** k, 0.99 * 448 * 2.0 ** k)
+        r[g.integers(0, 128)] = (448.0 if k % 2 else -448.0) * 2.0 ** k
+        rows.append(r)
+    x = _bf16_groups(rows)
+    q8, s8 = oracle_mod.quant_group128_ue8m0(x)
+    q32, s32 = oracle_mod.quant_group128(x)
+    assert np.array_equal(q8, q32)
+    assert np.array_equal(oracle_mod.e8m0_to_f32(s8), s32)
+
+
+def test_ue8m0_scale_is_tight_and_codes_round_trip(oracle_mod):
+    """amax * 2^-e lies in (224, 448] (the smallest power of two that fits), and
+    every code is within half an E4M3 step of x * 2^-e."""
+    x = inputs.bf16_bits(inputs.activations_group(64, k=1024))
+    q, s = oracle_mod.quant_group128_ue8m0(x)
+    xs = (x.astype(np.uint32) << 16).view(np.float32).astype(np.float64).reshape(64, 8, 128)
+    e = s.astype(np.int64) - 127
+    v = xs * np.ldexp(1.0, -e)[:, :, None]
+    am = np.abs(v).max(axis=2)
+    assert np.all((am > 224.0) & (am <= 448.0))
+    dec = oracle_mod.e4m3_decode(q).reshape(64, 8, 128)
+    mag = np.abs(v)
+    step = np.where(mag >= 2.0 ** -6, 2.0 ** (np.floor(np.log2(np.maximum(mag, 2.0 ** -6))) - 3), 2.0 ** -9)
+    assert np.all(np.abs(dec - v) <= step / 2)
+
+
+def test_ue8m0_special_groups(oracle_mod):
+    tiny = float(np.float32(2.0 ** -133))                  # smallest bf16 subnormal
+    x = _bf16_groups([[0.0] * 64 + [-0.0] * 64,
+                      [1.0] * 127 + [float("nan")],
+                      [2.0] * 127 + [float("-inf")],
+                      [tiny] * 128])
+    q, s = oracle_mod.quant_group128_ue8m0(x)
+    assert s[:, 0].tolist() == [0, 255, 255, 0]
+    assert set(q[0, :64].tolist()) == {0x00} and set(q[0, 64:].tolist()) == {0x80}
+    assert set(q[1].tolist()) == {0x7F} and set(q[2].tolist()) == {0x7F}
+    assert set(q[3].tolist()) == {0x08}                    # 2^-133 * 2^127 = 2^-6, the smallest normal
+
+
+def test_ue8m0_block128_is_group_rule_on_blocks(oracle_mod):
+    """Weight blocks: byte from the block's max |w| (numpy), codes of w * 2^-e."""
+    w = inputs.bf16_bits(inputs.weight_tiny())
+    q, s = oracle_mod.quant_block128_ue8m0(w)
+    n, k = w.shape
+    wf = (w.astype(np.uint32) << 16).view(np.float32)
+    for nb in range((n + 127) // 128):
+        for g in range(k // 128):
+            blk = wf[nb * 128:(nb + 1) * 128, g * 128:(g + 1) * 128]
+            assert s[nb, g] == oracle_mod.e8m0_from_amax(float(np.abs(blk).max()))
+            v = blk.astype(np.float64) * 2.0 ** (127 - int(s[nb, g]))
+            want = oracle_mod.e4m3_encode(v.astype(np.float32))
+            assert np.array_equal(q[nb * 128:(nb + 1) * 128, g * 128:(g + 1) * 128], want)
+
+
+def test_gemm_ue8m0_is_integer_matmul_times_powers_of_two(oracle_mod):
+    """R = sum_kb 2^(ea+eb) * (A_kb @ B_kb^T), each term exact in float64."""
+    qa, _, qb, _ = inputs.gemm_operands(9, 300, 512, seed=33)
+    g = np.random.default_rng(34)
+    sa = g.integers(100, 150, (9, 4)).astype(np.uint8)
+    sb = g.integers(100, 150, (3, 4)).astype(np.uint8)
+    R, _ = oracle_mod.gemm_ue8m0(qa, sa, qb, sb)
+    A = torch_decode(qa)
+    B = torch_decode(qb)
+    ref = np.zeros((9, 300))
+    for kb in range(4):
+        part = A[:, kb * 128:(kb + 1) * 128] @ B[:, kb * 128:(kb + 1) * 128].T
+        ea = sa[:, kb].astype(np.int64) - 127
+        eb = sb[np.arange(300) // 128, kb].astype(np.int64) - 127
+        ref += part * np.ldexp(1.0, ea[:, None] + eb[None, :])
+    assert np.array_equal(R, ref)
