@@ -24,7 +24,8 @@ from . import _abi
 
 __all__ = [
     "act_quant_per_tensor", "act_amax", "act_quant_apply", "act_quant_group128",
-    "weight_quant_block128", "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
+    "weight_quant_block128", "act_quant_group128_ue8m0", "weight_quant_block128_ue8m0",
+    "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
     "device_status",
     "per_tensor_sharded", "Fp8qError", "library",
 ]
@@ -140,6 +141,37 @@ def weight_quant_block128(w: torch.Tensor):
     s = torch.empty(((N + 127) // 128, K // 128), dtype=torch.float32, device=w.device)
     _abi.check(lib.fp8_weight_quant_block128(w.data_ptr(), N, K, ldw, q.data_ptr(), K, s.data_ptr(),
                                              _stream(w.device)), "fp8_weight_quant_block128")
+    return q.view(E4M3), s
+
+
+def act_quant_group128_ue8m0(x: torch.Tensor):
+    """Per-1x128-group quantisation with power-of-two (ue8m0) scales.
+
+    Returns (codes [M,K] float8_e4m3fn, E8M0 scale bytes [M,K/128] uint8;
+    scale value 2^(b-127), 255 = NaN)."""
+    lib = _abi.load()
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    M, K, ldx = _rows(x, "x")
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty((M, K // 128), dtype=torch.uint8, device=x.device)
+    _abi.check(lib.fp8_act_quant_group128_ue8m0(x.data_ptr(), M, K, ldx, q.data_ptr(), K, s.data_ptr(),
+                                                _stream(x.device)), "fp8_act_quant_group128_ue8m0")
+    return q.view(E4M3), s
+
+
+def weight_quant_block128_ue8m0(w: torch.Tensor):
+    """Per-128x128-block quantisation with power-of-two (ue8m0) scales.
+
+    Returns (codes [N,K] float8_e4m3fn, E8M0 bytes [ceil(N/128), K/128] uint8)."""
+    lib = _abi.load()
+    if w.dtype != torch.bfloat16:
+        raise TypeError("w must be bfloat16")
+    N, K, ldw = _rows(w, "w")
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    s = torch.empty(((N + 127) // 128, K // 128), dtype=torch.uint8, device=w.device)
+    _abi.check(lib.fp8_weight_quant_block128_ue8m0(w.data_ptr(), N, K, ldw, q.data_ptr(), K, s.data_ptr(),
+                                                   _stream(w.device)), "fp8_weight_quant_block128_ue8m0")
     return q.view(E4M3), s
 
 

@@ -502,13 +502,14 @@ int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
 }
 
 // ------------------------------------------------------------ group / block
-int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
-                           int64_t ldq, float* scales, void* stream) {
+// e8: ue8m0 scales (E8M0 bytes) instead of fp32 amax/448.
+static int run_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q, int64_t ldq,
+                        void* scales, bool e8, void* stream) {
     int rc = check_bf16_matrix(x, M, K, ldx, q, ldq, 128);
     if (rc != FP8Q_OK) return rc;
     if (M == 0 || K == 0) return FP8Q_OK;
     if (!scales) return FP8Q_ERR_INVALID_ARG;
-    if (!aligned4(scales)) return FP8Q_ERR_MISALIGNED;
+    if (!e8 && !aligned4(scales)) return FP8Q_ERR_MISALIGNED;
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d)) != FP8Q_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -518,31 +519,58 @@ int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uin
                          (int64_t(kQuantThreads) * kGroupU);
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(d->sms) * kBlocksPerSm)));
     if (log_enabled())
-        std::fprintf(stderr, "[fp8q] group128 M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
+        std::fprintf(stderr, "[fp8q] group128%s M=%lld K=%lld: grid=%d\n", e8 ? " ue8m0" : "",
+                     (long long)M, (long long)K, grid);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
-    if (ldx == K && ldq == K)
+    const bool contig = ldx == K && ldq == K;
+    if (e8 && contig)
+        group128_quant_kernel<kGroupU, true, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+    else if (e8)
+        group128_quant_kernel<kGroupU, false, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+    else if (contig)
         group128_quant_kernel<kGroupU, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
     else
         group128_quant_kernel<kGroupU, false><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
     return launch_status();
 }
 
-int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* qb,
-                              int64_t ldqb, float* sb, void* stream) {
+static int run_block128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* qb, int64_t ldqb,
+                        void* sb, bool e8, void* stream) {
     int rc = check_bf16_matrix(w, N, K, ldw, qb, ldqb, 128);
     if (rc != FP8Q_OK) return rc;
     if (N == 0 || K == 0) return FP8Q_OK;
     if (!sb) return FP8Q_ERR_INVALID_ARG;
-    if (!aligned4(sb)) return FP8Q_ERR_MISALIGNED;
+    if (!e8 && !aligned4(sb)) return FP8Q_ERR_MISALIGNED;
     if ((N + 127) / 128 > 65535) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     DeviceInfo* d = nullptr;
     if ((rc = device_info(&d)) != FP8Q_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t G = K / 128;
     dim3 grid(unsigned(G), unsigned((N + 127) / 128));
-    block128_quant_kernel<<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(w), N, ldw, qb,
-                                                          ldqb, sb, G);
+    const uint16_t* ws = static_cast<const uint16_t*>(w);
+    if (e8) block128_quant_kernel<true><<<grid, kQuantThreads, 0, st>>>(ws, N, ldw, qb, ldqb, sb, G);
+    else block128_quant_kernel<false><<<grid, kQuantThreads, 0, st>>>(ws, N, ldw, qb, ldqb, sb, G);
     return launch_status();
+}
+
+int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                           int64_t ldq, float* scales, void* stream) {
+    return run_group128(x, M, K, ldx, q, ldq, scales, false, stream);
+}
+
+int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* qb,
+                              int64_t ldqb, float* sb, void* stream) {
+    return run_block128(w, N, K, ldw, qb, ldqb, sb, false, stream);
+}
+
+int fp8_act_quant_group128_ue8m0(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                                 int64_t ldq, uint8_t* scales, void* stream) {
+    return run_group128(x, M, K, ldx, q, ldq, scales, true, stream);
+}
+
+int fp8_weight_quant_block128_ue8m0(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_t* qb,
+                                    int64_t ldqb, uint8_t* sb, void* stream) {
+    return run_block128(w, N, K, ldw, qb, ldqb, sb, true, stream);
 }
 
 // ------------------------------------------------------------ GEMM

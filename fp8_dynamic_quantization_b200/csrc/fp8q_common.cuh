@@ -134,6 +134,41 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, const Scale& d, bool exa
     return r;
 }
 
+// ---------------------------------------------------------------------------
+// ue8m0 scales: the scale is the smallest power of two 2^e >= amax/448 with
+// e clamped to [-127, 127], stored as the E8M0 byte e + 127 (255 = NaN).
+// For a normal bf16 amax = 1.f x 2^E, amax/448 = (1.f / 1.75) x 2^(E-8) and
+// 1.f / 1.75 lies in [4/7, 1] when the 7-bit fraction field is at most 0x60
+// (1.75) and in (1, 8/7) above it, so e = E - 8, plus 1 above 0x60.  Zero,
+// subnormal and small amax clamp to e = -127; Inf and NaN give 255.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e8m0_from_amax_bits(uint32_t m) {
+    if (m >= 0x7F80u) return 255u;
+    const int E = int(m >> 7) - 127;
+    const int e = max(E - 8 + ((m & 0x7Fu) > 0x60u ? 1 : 0), -127);
+    return uint32_t(e + 127);
+}
+
+// 2^-(b-127) as fp32 (b <= 247 for any finite bf16 amax, so 254 - b >= 7:
+// a normal number), NaN for b = 255.
+__device__ __forceinline__ float e8m0_inverse(uint32_t b) {
+    return b == 255u ? __uint_as_float(0x7FC00000u) : __uint_as_float((254u - b) << 23);
+}
+
+// Codes of 8 bf16 values for a power-of-two scale: e4m3_rne(x * 2^-e).  The
+// product is exact unless it falls below 2^-126, where every candidate
+// rounds to a signed-zero code anyway; |x| <= amax keeps it within +-448.
+__device__ __forceinline__ uint2 quant8_pow2(const uint4& v, float inv) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(__fmul_rn(bf16_lo(w[i]), inv), __fmul_rn(bf16_hi(w[i]), inv));
+    uint2 r;
+    r.x = c[0] | (c[1] << 16);
+    r.y = c[2] | (c[3] << 16);
+    return r;
+}
+
 // Streaming global accesses: read-only, no L1 allocation; stores evict-first.
 __device__ __forceinline__ uint4 ld_stream16(const void* p) {
     uint4 v;

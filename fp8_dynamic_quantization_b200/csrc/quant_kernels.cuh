@@ -20,6 +20,8 @@
 //                            cluster; values stay in registers while the
 //                            CTAs exchange partial maxima on chip.
 //  block128_quant_kernel     128x128 weight blocks (offline step).
+//  Both group and block kernels also have a ue8m0 form (E8 = true): the
+//  scale is the smallest power of two >= amax/448, written as an E8M0 byte.
 #pragma once
 
 #include "fp8q_common.cuh"
@@ -46,11 +48,12 @@ __device__ __forceinline__ int64_t vec_offset(int64_t i, int64_t vec_per_row, in
 // values per thread.  Each thread carries U groups per iteration (2U loads
 // in flight).
 // ---------------------------------------------------------------------------
-template <int U, bool CONTIG>
+// E8: ue8m0 scales (E8M0 bytes in `scales`) instead of fp32 amax/448.
+template <int U, bool CONTIG, bool E8 = false>
 __global__ void __launch_bounds__(kQuantThreads)
 group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                       uint8_t* __restrict__ q, int64_t ldq,
-                      float* __restrict__ scales, int64_t groups, int64_t G) {
+                      void* __restrict__ scales, int64_t groups, int64_t G) {
     const int sub = threadIdx.x & 7;
     const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 3;
     const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 3;
@@ -81,11 +84,21 @@ group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
             m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-            const Scale d = make_scale(scale_from_amax_bits(m));
-            if (g < groups) {
-                st_stream8(q + qo[u], quant8(a[u], d));
-                st_stream8(q + qo[u] + 64, quant8(b[u], d));
-                if (sub == 0) scales[g] = d.s;
+            if (E8) {
+                const uint32_t sb = e8m0_from_amax_bits(m);
+                const float inv = e8m0_inverse(sb);
+                if (g < groups) {
+                    st_stream8(q + qo[u], quant8_pow2(a[u], inv));
+                    st_stream8(q + qo[u] + 64, quant8_pow2(b[u], inv));
+                    if (sub == 0) static_cast<uint8_t*>(scales)[g] = uint8_t(sb);
+                }
+            } else {
+                const Scale d = make_scale(scale_from_amax_bits(m));
+                if (g < groups) {
+                    st_stream8(q + qo[u], quant8(a[u], d));
+                    st_stream8(q + qo[u] + 64, quant8(b[u], d));
+                    if (sub == 0) static_cast<float*>(scales)[g] = d.s;
+                }
             }
         }
     }
@@ -255,9 +268,10 @@ __global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float*
 // thread keeps its 8 vectors in registers between the amax and the apply.
 // grid = (K/128, ceil(N/128)).
 // ---------------------------------------------------------------------------
+template <bool E8 = false>   // E8: E8M0 scale bytes in `sb` (ue8m0 variant)
 __global__ void __launch_bounds__(kQuantThreads)
 block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
-                      uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ sb, int64_t G) {
+                      uint8_t* __restrict__ q, int64_t ldq, void* __restrict__ sb, int64_t G) {
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t kb = blockIdx.x, nb = blockIdx.y;
     uint4 v[8];
@@ -271,8 +285,21 @@ block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
         m = max(m, absmax8(v[u]));
     }
     m = block_max<kQuantThreads>(m, red);
+    if (E8) {
+        const uint32_t b = e8m0_from_amax_bits(m);
+        const float inv = e8m0_inverse(b);
+        if (threadIdx.x == 0) static_cast<uint8_t*>(sb)[nb * G + kb] = uint8_t(b);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int j = threadIdx.x + u * kQuantThreads;
+            const int64_t r = nb * 128 + (j >> 4);
+            const int c = (j & 15) * 8;
+            if (r < N) st_stream8(q + r * ldq + kb * 128 + c, quant8_pow2(v[u], inv));
+        }
+        return;
+    }
     const Scale d = make_scale(scale_from_amax_bits(m));
-    if (threadIdx.x == 0) sb[nb * G + kb] = d.s;
+    if (threadIdx.x == 0) static_cast<float*>(sb)[nb * G + kb] = d.s;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
         const int j = threadIdx.x + u * kQuantThreads;

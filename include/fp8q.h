@@ -147,6 +147,27 @@ int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw,
                               uint8_t* qb, int64_t ldqb, float* sb, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* ue8m0 (power-of-two) scales ([P1] Benchmarking the Activation        */
+/* Quantization Kernel: act_quant(..., scale_fmt="ue8m0")).  The page   */
+/* names the format only.  Reading: the scale is the smallest power of  */
+/* two 2^e >= amax/448, e clamped to [-127, 127], stored as the E8M0    */
+/* byte e + 127 (value 2^(b-127); 255 = NaN).  An all-zero group gets   */
+/* byte 0; an Inf or NaN amax gives byte 255 and NaN codes (0x7F).      */
+/* Codes are e4m3_rne(x * 2^-e): x * 2^-e is exact, so the one rounding  */
+/* is the conversion, and |x * 2^-e| <= 448 means nothing saturates.     */
+/* ------------------------------------------------------------------ */
+
+/* As fp8_act_quant_group128, with E8M0 scale bytes: scales[m*(K/128)+g]
+ * (uint8, contiguous).  No alignment requirement on scales. */
+int fp8_act_quant_group128_ue8m0(const void* x, int64_t M, int64_t K, int64_t ldx,
+                                 uint8_t* q, int64_t ldq, uint8_t* scales, void* stream);
+
+/* As fp8_weight_quant_block128, with E8M0 scale bytes sb[nb*(K/128)+kb]
+ * (uint8, [ceil(N/128), K/128] contiguous). */
+int fp8_weight_quant_block128_ue8m0(const void* w, int64_t N, int64_t K, int64_t ldw,
+                                    uint8_t* qb, int64_t ldqb, uint8_t* sb, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Block-scaled FP8 GEMM ([P1] FP8 GEMM with per-block scaling,         */
 /* BLOCK_SIZE_K = 128)                                                  */
 /* ------------------------------------------------------------------ */
