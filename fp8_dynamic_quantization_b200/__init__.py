@@ -25,6 +25,7 @@ from . import _abi
 __all__ = [
     "act_quant_per_tensor", "act_amax", "act_quant_apply", "act_quant_group128",
     "weight_quant_block128", "act_quant_group128_ue8m0", "weight_quant_block128_ue8m0",
+    "block_gemm_ue8m0", "linear_ue8m0",
     "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
     "device_status",
     "per_tensor_sharded", "Fp8qError", "library",
@@ -243,6 +244,42 @@ def linear_per_tensor(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> to
     weight codes qb with scale sb."""
     qa, sa = act_quant_per_tensor(x)
     return gemm_per_tensor(qa, sa, qb, sb)
+
+
+def block_gemm_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 Y[M,N] = A * B^T with E8M0 (power-of-two) block scales, applied
+    by the tensor cores: sa uint8 [M,K/128], sb uint8 [ceil(N/128),K/128]."""
+    lib = _abi.load()
+    M, K, lda = _rows(_codes(qa, "qa"), "qa")
+    N, Kb, ldb = _rows(_codes(qb, "qb"), "qb")
+    if K != Kb:
+        raise ValueError("qa and qb must share K")
+    if sa.dtype != torch.uint8 or tuple(sa.shape) != (M, K // 128) or not sa.is_contiguous():
+        raise ValueError("sa must be a contiguous uint8 [M, K/128] tensor")
+    if sb.dtype != torch.uint8 or tuple(sb.shape) != ((N + 127) // 128, K // 128) or not sb.is_contiguous():
+        raise ValueError("sb must be a contiguous uint8 [ceil(N/128), K/128] tensor")
+    if out is None:
+        ldy_alloc = (N + 7) // 8 * 8
+        out = torch.empty((M, ldy_alloc), dtype=torch.bfloat16, device=qa.device)[:, :N]
+    _, _, ldy = _rows(out, "out")
+    nbytes = lib.fp8_block_gemm_workspace_size(M, N, K)
+    ws_ptr, ws_len = None, 0
+    if nbytes:
+        ws = _workspace("gemm", qa.device, nbytes, zero=False)
+        ws_ptr, ws_len = ws.data_ptr(), ws.numel()
+    _abi.check(lib.fp8_block_gemm_ue8m0(qa.data_ptr(), lda, sa.data_ptr(), qb.data_ptr(), ldb, sb.data_ptr(),
+                                        out.data_ptr(), ldy, M, N, K, ws_ptr, ws_len, _stream(qa.device)),
+               "fp8_block_gemm_ue8m0")
+    return out
+
+
+def linear_ue8m0(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:
+    """The dynamic FP8 linear method with ue8m0 scales: group-128 quantise x
+    with power-of-two scales, then the block-scaled GEMM against weight codes
+    qb with E8M0 block scales sb."""
+    qa, sa = act_quant_group128_ue8m0(x)
+    return block_gemm_ue8m0(qa, sa, qb, sb)
 
 
 def linear(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:

@@ -52,11 +52,11 @@ constexpr int kStreamU = 4;         // vectors per thread per iteration elsewher
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 cudaError_t set_gemm_smem() {
-    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT, SS>,
+    return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                int(GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>::kSmemBytes));
+                                int(GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>::kSmemBytes));
 }
 
 // Device facts, queried once per device.  FP8Q_ERR_NO_DEVICE unless the
@@ -98,6 +98,13 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, 2>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, 2>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, true>();
                 if (e != cudaSuccess) { cudaGetLastError(); d.status = FP8Q_ERR_CUDA; }
             }
@@ -203,9 +210,9 @@ bool tile_override(TableRow* out) {
     return has;
 }
 
-// The per-tensor GEMM has no CTA-pair variant: a forced pair row runs as the
-// single-CTA tile of the same width.
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool per_tensor = false) {
+// Only the fp32 block-scaled GEMM has a CTA-pair variant: for the others a
+// forced pair row runs as the single-CTA tile of the same width.
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = false) {
     GemmPlan pl{};
     const TableRow* row = &kGemmTable[0];
     for (const TableRow& r : kGemmTable)
@@ -213,7 +220,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool per_tensor = f
     TableRow forced;
     if (tile_override(&forced)) row = &forced;
     pl.swap = row->mode == kSwap;
-    pl.pair = row->mode == kPair && !per_tensor;
+    pl.pair = row->mode == kPair && !no_pair;
     pl.bn = row->bn;
     pl.stages = pl.swap ? (pl.bn == 16 ? 12 : pl.bn == 32 ? 10 : pl.bn == 64 ? 8 : 6)
                         : pl.pair ? (pl.bn == 256 ? 6 : 8) : (pl.bn == 192 ? 5 : pl.bn == 256 ? 4 : 6);
@@ -292,12 +299,12 @@ bool make_scale_tmap(CUtensorMap* m, const float* base, int64_t rows, int64_t G,
 }
 
 // tsa/tsb: scale maps (staged-scale variants only; the others ignore them)
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& tsa, const CUtensorMap& tsb,
                  const GemmParams& p, int grid, cudaStream_t st) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>;
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
     if (!PAIR) {
-        block_gemm_kernel<BN, SWAP, STAGES, PAIR, PT, SS><<<grid, C::kThreads, C::kSmemBytes, st>>>(
+        block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS><<<grid, C::kThreads, C::kSmemBytes, st>>>(
             tp, tq, tsa, tsb, p);
         return;
     }
@@ -585,7 +592,9 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                    void* workspace, size_t workspace_bytes, void* stream, bool per_tensor) {
+                    void* workspace, size_t workspace_bytes, void* stream, int mode) {
+    // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes
+    const bool per_tensor = mode == 1, ue8m0 = mode == 2;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
@@ -593,7 +602,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     if (!qa || !sa || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
     if (lda < K || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
     if (!aligned16(qa) || !aligned16(qb) || !aligned16(y) || lda % 16 || ldb % 16 || (ldy * 2) % 16 ||
-        !aligned4(sa) || !aligned4(sb))
+        (!ue8m0 && (!aligned4(sa) || !aligned4(sb))))
         return FP8Q_ERR_MISALIGNED;
     DeviceInfo* d = nullptr;
     int rc = device_info(&d);
@@ -604,7 +613,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, per_tensor);
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode != 0);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -631,7 +640,8 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     p.tiles_q = pl.tiles_q;
     p.splits = pl.splits;
     p.units = pl.units;
-    p.scale_vec4 = !per_tensor && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
+    p.scale_vec4 = mode == 0 && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
+    p.sf_words = ue8m0 && (p.G % 4 == 0) && aligned4(sa) && aligned4(sb);
     // Normal 128/256-wide tiles stage the block scales through shared memory
     // (TMA boxes of 4 K blocks) when the scale rows allow 16-byte boxes.
     const bool staged = p.scale_vec4 && !pl.swap && !pl.pair && (pl.bn == 128 || pl.bn == 256);
@@ -645,7 +655,22 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
-    if (per_tensor) {
+    if (ue8m0) {
+        if (pl.swap) {
+            switch (pl.bn) {
+                case 16: launch_gemm<16, true, 12, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 32: launch_gemm<32, true, 10, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 64: launch_gemm<64, true, 8, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                default: launch_gemm<128, true, 6, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+            }
+        } else if (pl.bn == 128) {
+            launch_gemm<128, false, 6, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else if (pl.bn == 192) {
+            launch_gemm<192, false, 5, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else {
+            launch_gemm<256, false, 4, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st);
+        }
+    } else if (per_tensor) {
         if (pl.swap) {
             switch (pl.bn) {
                 case 16: launch_gemm<16, true, 12, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
@@ -692,13 +717,20 @@ extern "C" {
 int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                    const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                    void* workspace, size_t workspace_bytes, void* stream) {
-    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, false);
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 0);
 }
 
 int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                         const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream) {
-    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, true);
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 1);
+}
+
+int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa, const uint8_t* qb, int64_t ldb,
+                         const uint8_t* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    return run_gemm(qa, lda, reinterpret_cast<const float*>(sa), qb, ldb, reinterpret_cast<const float*>(sb),
+                    y, ldy, M, N, K, workspace, workspace_bytes, stream, 2);
 }
 
 // ------------------------------------------------------------ GEMM, no allocation

@@ -37,10 +37,22 @@
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
 //
-// PT (per-tensor scales, the GEMM of the per-tensor dynamic path): sa and sb
-// are single fp32 values, so no per-block promotion is needed -- the MMAs
-// accumulate a unit's whole K range into one TMEM buffer and the epilogue
-// multiplies it by sa*sb once.
+// Scale mode SM:
+//   0  fp32 block scales, promoted per K block as above.
+//   1  per-tensor scales (the GEMM of the per-tensor dynamic path): sa and
+//      sb are single fp32 values, so the MMAs accumulate a unit's whole K
+//      range into one TMEM buffer and the epilogue multiplies by sa*sb once.
+//   2  ue8m0 block scales (E8M0 bytes sa [M, G], sb [ceil(N/128), G]): the
+//      tensor cores apply them (tcgen05.mma kind::mxf8f6f4.block_scale), so
+//      again one TMEM accumulation per unit and no promotion.  Per group of 4
+//      K blocks the producer warp writes the tile's scale bytes into a
+//      shared-memory slot laid out as 32 rows x 16 bytes per 128 rows
+//      (row j holds rows j, 32+j, 64+j, 96+j, four K blocks each); the MMA
+//      warp copies each such block to TMEM with tcgen05.cp 32x128b.warpx4,
+//      which replicates it into all four lane quarters -- the layout the
+//      block-scaled MMA reads: A row m at lane m, column base + m/32; B row n
+//      at column base + n/32 in every lane quarter; the byte picked by the
+//      instruction's scale-factor id, here kb % 4.
 #pragma once
 
 #include <cuda.h>
@@ -58,11 +70,14 @@ struct GemmParams {
     int M, N, G;
     int tiles_p, tiles_q, splits, units;
     int scale_vec4;      // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
+    int sf_words;        // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 struct GemmCfg {
+    static constexpr bool PT = SM == 1;                        // per-tensor scales
+    static constexpr bool MX = SM == 2;                        // ue8m0 scales applied by the MMA
     // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
     // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
     // and its TMEM receives its 128 rows x BN columns of every product.
@@ -82,11 +97,17 @@ struct GemmCfg {
     static constexpr int kQRows = PAIR ? BN / 2 : BN;         // B (or A) rows this CTA loads
     static constexpr int kQBytes = kQRows * 128;
     static constexpr int kStageBytes = kPBytes + kQBytes;
-    static constexpr int kNumBuf = (512 / BN) < 8 ? (512 / BN) : 8;
-    static constexpr int kTmemCols = kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
+    // MX keeps TMEM columns [448, 512) for four scale-factor slots of 16
+    // columns (B scales at +0..7, A scales at +8..11).
+    static constexpr int kSfSlots = MX ? 4 : 0;
+    static constexpr int kSfCol0 = 448;
+    static constexpr int kSfSlotBytes = 3 * 512;               // A block, B rows 0-127, B rows 128-255
+    static constexpr int kDataCols = MX ? kSfCol0 : 512;
+    static constexpr int kNumBuf = (kDataCols / BN) < 8 ? (kDataCols / BN) : 8;
+    static constexpr int kTmemCols = MX ? 512 : kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
     static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
-    static constexpr int kSlabFloats = (SWAP && !PT) ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
+    static constexpr int kSlabFloats = (SWAP && SM == 0) ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
     // SS: block scales staged through shared memory.  The producer copies,
     // per group of 4 K blocks, the tile's 128 x 4 row scales and its
     // BN/128 x 4 column-block scales into a ring of kScaleSlots slots.
@@ -95,7 +116,8 @@ struct GemmCfg {
     static constexpr int kScaleSlotBytes = 2048 + 128;         // 128 x 4 fp32, then kSbRows x 4 fp32
     static constexpr uint32_t kScaleTx = 2048 + 16 * kSbRows;  // bytes one slot receives
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
-                                         + size_t(kSlabFloats) * 4 + size_t(kScaleSlots) * kScaleSlotBytes + 512;
+                                         + size_t(kSlabFloats) * 4 + size_t(kScaleSlots) * kScaleSlotBytes
+                                         + size_t(kSfSlots) * kSfSlotBytes + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(kCW % 16 == 0, "columns per thread");
     static_assert(!SWAP || BN <= 128, "swapped tiles hold at most 128 tokens");
@@ -105,8 +127,9 @@ struct GemmCfg {
     static_assert(!PAIR || (!SWAP && (BN == 256 || BN == 128)), "CTA pairs compute 256 x 256 or 256 x 128 tiles");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kSmemBytes <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * kNumBuf + 2 * kScaleSlots) * 8 + 8 <= 512, "barrier area");
-    static_assert(!SS || (!SWAP && !PAIR && !PT && (BN == 128 || BN == 256)), "staged scales: normal 128/256 tiles");
+    static_assert((2 * STAGES + 2 * kNumBuf + 2 * kScaleSlots + 2 * kSfSlots) * 8 + 8 <= 512, "barrier area");
+    static_assert(!SS || (!SWAP && !PAIR && SM == 0 && (BN == 128 || BN == 256)), "staged scales: normal 128/256 tiles");
+    static_assert(!MX || (!PAIR && kNumBuf >= 1), "ue8m0 tiles: one CTA, at least one TMEM buffer");
 };
 
 __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp, int& tq,
@@ -155,30 +178,86 @@ __device__ __forceinline__ float pick4(const float4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
-template <int BN, bool SWAP, int STAGES, bool PAIR = false, bool PT = false, bool SS = false>
-__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>::kThreads, 1)
+// ue8m0 mode: E8M0 bytes of K blocks [4g, 4g+4) for one 128-row block of
+// the P operand (is_p) or the Q operand, packed 4 per word (K block 4g+b in
+// byte b); rows, blocks and K blocks out of range give 127 (scale 1).
+template <int BN, bool SWAP>
+__device__ __forceinline__ uint32_t sf_word(const GemmParams& p, bool is_p, int tp, int tq, int row, int g) {
+    const uint8_t* sa = reinterpret_cast<const uint8_t*>(p.sa);   // [M, G]
+    const uint8_t* sb = reinterpret_cast<const uint8_t*>(p.sb);   // [ceil(N/128), G]
+    int64_t base = -1;                                            // byte offset of K block 0
+    if (is_p) {
+        if (!SWAP) { const int m = tp * 128 + row; if (m < p.M) base = int64_t(m) * p.G; }
+        else base = int64_t(tp) * p.G;                            // one weight block per P tile
+    } else {
+        if (!SWAP) { const int n = tq * BN + row; if (row < BN && n < p.N) base = int64_t(n >> 7) * p.G; }
+        else { const int m = tq * BN + row; if (row < BN && m < p.M) base = int64_t(m) * p.G; }
+    }
+    const uint8_t* src = (is_p != SWAP) ? sa : sb;
+    if (p.sf_words) {                       // K blocks 4g..4g+3 are bytes 0..3 of one aligned word
+        return base >= 0 ? __ldg(reinterpret_cast<const uint32_t*>(src + base + 4 * g)) : 0x7F7F7F7Fu;
+    }
+    uint32_t w = 0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+        const int kb = 4 * g + b;
+        const uint32_t v = (base >= 0 && kb < p.G) ? uint32_t(__ldg(src + base + kb)) : 127u;
+        w |= v << (8 * b);
+    }
+    return w;
+}
+
+// One scale slot: the A block (P rows) and ceil(BN/128) B blocks, each 32
+// rows x 16 bytes; lane j writes row j of every block.
+template <int BN, bool SWAP>
+__device__ __forceinline__ void build_sf_slot(uint8_t* dst, const GemmParams& p, int lane, int tp, int tq, int g) {
+    uint4 a;
+    a.x = sf_word<BN, SWAP>(p, true, tp, tq, lane, g);
+    a.y = sf_word<BN, SWAP>(p, true, tp, tq, 32 + lane, g);
+    a.z = sf_word<BN, SWAP>(p, true, tp, tq, 64 + lane, g);
+    a.w = sf_word<BN, SWAP>(p, true, tp, tq, 96 + lane, g);
+    *reinterpret_cast<uint4*>(dst + lane * 16) = a;
+#pragma unroll
+    for (int blk = 0; blk < (BN + 127) / 128; ++blk) {
+        uint4 b;
+        b.x = sf_word<BN, SWAP>(p, false, tp, tq, 128 * blk + lane, g);
+        b.y = sf_word<BN, SWAP>(p, false, tp, tq, 128 * blk + 32 + lane, g);
+        b.z = sf_word<BN, SWAP>(p, false, tp, tq, 128 * blk + 64 + lane, g);
+        b.w = sf_word<BN, SWAP>(p, false, tp, tq, 128 * blk + 96 + lane, g);
+        *reinterpret_cast<uint4*>(dst + 512 * (1 + blk) + lane * 16) = b;
+    }
+}
+
+template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
+__global__ void __launch_bounds__(GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>::kThreads, 1)
 block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmSA,    // row scales [M, G] fp32 (SS only)
                   const __grid_constant__ CUtensorMap tmSB,    // column-block scales [NB, G] fp32 (SS only)
                   const GemmParams p) {
-    using C = GemmCfg<BN, SWAP, STAGES, PAIR, PT, SS>;
+    using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
+    constexpr bool PT = C::PT, MX = C::MX;
+    constexpr bool ONE = PT || MX;        // one TMEM accumulation per unit, no per-K-block promotion
     constexpr int NB = C::kNumBuf;
     constexpr uint32_t kSlots = C::kScaleSlots > 0 ? C::kScaleSlots : 1;   // divisor for the (SS) slot ring
+    constexpr uint32_t kSfN = C::kSfSlots > 0 ? C::kSfSlots : 1;         // divisor for the (MX) slot ring
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* tiles = smem;                                        // STAGES x (P | Q)
     float* slab = reinterpret_cast<float*>(smem + size_t(STAGES) * C::kStageBytes);
     uint8_t* sring = smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4;   // SS slots
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sring + size_t(C::kScaleSlots) * C::kScaleSlotBytes);
+    uint8_t* sfring = sring + size_t(C::kScaleSlots) * C::kScaleSlotBytes;   // MX scale-factor slots
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sfring + size_t(C::kSfSlots) * C::kSfSlotBytes);
     uint64_t* full = bars;                        // [STAGES] TMA landed
     uint64_t* empty = bars + STAGES;              // [STAGES] MMA done reading
     uint64_t* tfull = bars + 2 * STAGES;          // [NB] block partial ready in TMEM
     uint64_t* tempty = bars + 2 * STAGES + NB;    // [NB] promotion done reading TMEM
     uint64_t* sfull = bars + 2 * STAGES + 2 * NB;  // [kScaleSlots] scale slot landed (SS)
     uint64_t* sempty = sfull + C::kScaleSlots;     // [kScaleSlots] scale slot read by every promotion warp
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(sempty + C::kScaleSlots);
+    uint64_t* sffull = sempty + C::kScaleSlots;   // [kSfSlots] scale-factor slot written (MX)
+    uint64_t* sfempty = sffull + C::kSfSlots;     // [kSfSlots] slot consumed by the MMAs (MX)
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(sfempty + C::kSfSlots);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -197,6 +276,10 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         for (int i = 0; i < C::kScaleSlots; ++i) {
             ptx::mbar_init(&sfull[i], 1);
             ptx::mbar_init(&sempty[i], 4 * C::kEpiWG);
+        }
+        for (int i = 0; i < C::kSfSlots; ++i) {
+            ptx::mbar_init(&sffull[i], 1);
+            ptx::mbar_init(&sfempty[i], 1);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -220,7 +303,33 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 
     if (warp < 4) {
         if (C::kEpiWG > 1) ptx::regs_dec<C::kRegWG0>();
-        if (warp == 0 && lane == 0) {
+        if (MX && warp == 2) {
+            // ------------------------------------ scale-slot writer (ue8m0)
+            // All lanes write one slot per group of 4 K blocks, in the order
+            // the MMA warp consumes them; wait results are broadcast from
+            // lane 0 so the warp stays converged and stops together.
+            uint32_t sg = 0;
+            bool stop = false;
+            for (int u = unit0; u < p.units && !stop; u += unit_step) {
+                int tp, tq, kb0, kb1;
+                unit_coords(p, u, tp, tq, kb0, kb1);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (kb != kb0 && (kb & 3) != 0) continue;
+                    const uint32_t slot = sg % kSfN, sph = (sg / kSfN) & 1;
+                    bool ok = true;
+                    if (lane == 0) ok = ptx::mbar_wait(&sfempty[slot], sph ^ 1, p.wait_budget);
+                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                    if (!ok) { if (lane == 0) fail(); stop = true; break; }
+                    __syncwarp();
+                    build_sf_slot<BN, SWAP>(sfring + size_t(slot) * C::kSfSlotBytes, p, lane, tp, tq, kb >> 2);
+                    ptx::fence_proxy_async_shared();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(&sffull[slot]);
+                    ++sg;
+                }
+            }
+            __syncwarp();
+        } else if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- producer
             uint32_t it = 0;
             uint32_t sg = 0;             // scale groups issued (SS)
@@ -271,6 +380,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             // -------------------------------------------------------- MMA issuer
             constexpr uint32_t idesc = ptx::idesc_e4m3_f32(BN, C::kTileRows);
             uint32_t it = 0, c = 0;
+            uint32_t sgm = 0, sf_slot = 0, sf_col = 0;   // scale-factor slots (MX)
             bool failed = false;
             // the most recent commit (a commit arrives once every MMA issued
             // before it has finished): what an abort must wait for
@@ -282,7 +392,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 // One promotion step = one K block (block scales), or the
                 // whole K range of the unit (per-tensor scales: the MMAs
                 // accumulate every K block into one TMEM buffer).
-                const int steps = PT ? 1 : kb1 - kb0;
+                const int steps = ONE ? 1 : kb1 - kb0;
                 int kb = kb0;
                 for (int st = 0; st < steps && !failed; ++st, ++c) {
                     const uint32_t buf = c % NB, tph = (c / NB) & 1;
@@ -290,16 +400,37 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                                             : ptx::mbar_wait(&tempty[buf], tph ^ 1, p.wait_budget);
                     if (!freed) { fail(); failed = true; break; }
                     const uint32_t d = tmem_base + buf * BN;
-                    const int kb_end = PT ? kb1 : kb + 1;
+                    const int kb_end = ONE ? kb1 : kb + 1;
                     for (; kb < kb_end; ++kb, ++it) {
+                        if (MX && (kb == kb0 || (kb & 3) == 0)) {
+                            // this group's scale bytes: shared slot -> TMEM slot
+                            sf_slot = sgm % kSfN;
+                            const uint32_t sph = (sgm / kSfN) & 1;
+                            if (!ptx::mbar_wait(&sffull[sf_slot], sph, p.wait_budget)) { fail(); failed = true; break; }
+                            ptx::tc_fence_after();
+                            const uint32_t src = ptx::smem_u32(sfring + size_t(sf_slot) * C::kSfSlotBytes);
+                            sf_col = tmem_base + C::kSfCol0 + sf_slot * 16;
+                            ptx::tmem_cp_32x128b_x4(sf_col + 8, ptx::sf_block_desc(src));          // A
+                            ptx::tmem_cp_32x128b_x4(sf_col, ptx::sf_block_desc(src + 512));        // B rows 0-127
+                            if (BN > 128) ptx::tmem_cp_32x128b_x4(sf_col + 4, ptx::sf_block_desc(src + 1024));
+                            ++sgm;
+                        }
                         const int s = it % STAGES;
                         const uint32_t ph = (it / STAGES) & 1;
                         if (!ptx::mbar_wait(&full[s], ph, p.wait_budget)) { fail(); failed = true; break; }
                         ptx::tc_fence_after();
                         const uint32_t pa = ptx::smem_u32(tiles + size_t(s) * C::kStageBytes);
                         const uint32_t qa = pa + C::kPBytes;
-                        const uint32_t first = (PT && kb > kb0) ? 1u : 0u;   // accumulate across K blocks
-                        if (PAIR) {
+                        const uint32_t first = (ONE && kb > kb0) ? 1u : 0u;  // accumulate across K blocks
+                        if (MX) {
+                            const uint32_t idx = ptx::idesc_mx_e4m3(BN, uint32_t(kb & 3));
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                ptx::mma_f8_mx(d, ptx::sw128_kmajor_desc(pa + 32 * k), ptx::sw128_kmajor_desc(qa + 32 * k),
+                                               idx, sf_col + 8, sf_col, first | (k > 0));
+                            ptx::mma_commit(&empty[s]);
+                            if ((kb & 3) == 3 || kb == kb1 - 1) ptx::mma_commit(&sfempty[sf_slot]);
+                        } else if (PAIR) {
 #pragma unroll
                             for (int k = 0; k < 4; ++k)
                                 ptx::mma_f8_pair(d, ptx::sw128_kmajor_desc(pa + 32 * k),
@@ -354,7 +485,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             const int q0 = tq * BN;
             const int m_row = tp * C::kTileRows + int(rank) * 128 + row;   // normal: token row
             const int n_row = tp * 128 + row;                              // swapped: weight row
-            if (SWAP && !PT) {
+            if (SWAP && SM == 0) {
                 // slab[kbl*BN + j] = sa[q0+j, kb0+kbl] * sb[tp, kb0+kbl]
                 ptx::named_bar_sync(1, nthreads);
                 for (int i = etid; i < nkb * BN; i += nthreads) {
@@ -373,12 +504,12 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             // Normal mode: row scale sa[m_row, kb] times the column block's
             // sb[nb, kb], fetched four K blocks at a time, one group ahead.
             const int nb = (q0 + chalf * C::kCW) >> 7;
-            const bool row_ok = !SWAP && !PT && m_row < p.M;
-            const bool col_ok = !SWAP && !PT && nb * 128 < p.N;
+            const bool row_ok = !SWAP && SM == 0 && m_row < p.M;
+            const bool col_ok = !SWAP && SM == 0 && nb * 128 < p.N;
             const float* sa_row = p.sa + int64_t(SWAP ? 0 : (row_ok ? m_row : 0)) * p.G;
             const float* sb_row = p.sb + int64_t(col_ok ? nb : 0) * p.G;
             float4 sa_cur, sb_cur, sa_nxt, sb_nxt;
-            if (!SWAP && !PT && !SS) {
+            if (!SWAP && SM == 0 && !SS) {
                 sa_cur = load_scale4(sa_row, kb0 >> 2, p.G, vec4, row_ok);
                 sb_cur = load_scale4(sb_row, kb0 >> 2, p.G, vec4, col_ok);
                 sa_nxt = load_scale4(sa_row, (kb0 >> 2) + 1, p.G, vec4, row_ok);
@@ -386,8 +517,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             }
             bool ok = true;
             // per-tensor scales: one step per unit, one scalar scale
-            const int kb_last = PT ? kb0 + 1 : kb1;
-            const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : 0.0f;
+            const int kb_last = ONE ? kb0 + 1 : kb1;
+            const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : MX ? 1.0f : 0.0f;
             for (int kb = kb0; kb < kb_last; ++kb, ++c) {
                 float s = s_pt;
                 if (SS) {
@@ -404,7 +535,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                         ++sg;
                     }
                     s = pick4(sa_cur, kb & 3) * pick4(sb_cur, kb & 3);
-                } else if (!SWAP && !PT) {
+                } else if (!SWAP && SM == 0) {
                     if ((kb & 3) == 0 && kb != kb0) {
                         sa_cur = sa_nxt;
                         sb_cur = sb_nxt;
@@ -440,7 +571,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                             else ptx::mbar_arrive(&tempty[buf]);
                         }
                     }
-                    if (SWAP && !PT) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
+                    if (SWAP && SM == 0) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
                     else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
                 }
             }

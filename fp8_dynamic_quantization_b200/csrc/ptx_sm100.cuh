@@ -186,6 +186,54 @@ __device__ __forceinline__ void mma_f8_pair(uint32_t d_tmem, uint64_t a_desc, ui
         :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate) : "memory");
 }
 
+// D[tmem] (+)= (A * 2^sfa) * (B * 2^sfb)^T: E4M3 x E4M3 -> fp32 with E8M0
+// block scales read from TMEM (sfa_tmem / sfb_tmem; one scale per row per
+// 32 K; the byte of each 32-bit scale cell is chosen by the scale-factor ids
+// in idesc).
+__device__ __forceinline__ void mma_f8_mx(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+        :: "r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+        : "memory");
+}
+
+// Copy a 32-row x 16-byte shared-memory block to TMEM columns [taddr,
+// taddr+4) of lanes j, 32+j, 64+j and 96+j (row j; byte k in column k/4).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t desc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" :: "r"(taddr), "l"(desc) : "memory");
+}
+
+// Shared-memory descriptor of such a block: 16-byte rows, contiguous (no
+// swizzle; 8-row groups 128 bytes apart).
+__device__ __forceinline__ uint64_t sf_block_desc(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= uint64_t((saddr >> 4) & 0x3FFF);        // start address
+    d |= uint64_t(128 >> 4) << 32;               // stride byte offset
+    d |= uint64_t(1) << 46;                      // descriptor version
+    return d;                                    // layout 0: no swizzle
+}
+
+// Instruction descriptor of the block-scaled MMA: E4M3 x E4M3, both K-major,
+// E8M0 scales, M = 128, N = n; sf_id picks the byte of the A and B scale
+// cells.
+__host__ __device__ constexpr uint32_t idesc_mx_e4m3(int n, uint32_t sf_id) {
+    return (sf_id << 4)                    // B scale-factor id
+         | (0u << 7) | (0u << 10)          // A, B: E4M3
+         | (uint32_t(n >> 3) << 17)        // N / 8
+         | (1u << 23)                      // scale format E8M0
+         | (8u << 24)                      // M / 16 = 128 / 16
+         | (sf_id << 29);                  // A scale-factor id
+}
+
+// Make this thread's generic-proxy shared-memory writes visible to the
+// async proxy (tcgen05.cp, TMA) before it signals them.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Arrive once on the mbarrier at shared::cluster address `bar_cluster`
 // (this CTA's or the peer's) when the pair MMAs issued so far complete.
 __device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {

@@ -138,9 +138,26 @@ def run_gemm_pt(t, dev, m, n, k, reps, modes, hbm, fp8):
               "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
 
 
+def run_gemm_ue8m0(t, dev, m, n, k, reps, modes, hbm, fp8):
+    qa, _, qb, _ = inputs.gemm_operands(m, n, k)
+    g = np.random.default_rng(m + n)
+    tqa = torch.from_numpy(qa).to(dev).view(torch.float8_e4m3fn)
+    tqb = torch.from_numpy(qb).to(dev).view(torch.float8_e4m3fn)
+    sa = torch.from_numpy(g.integers(115, 135, (m, k // 128)).astype(np.uint8)).to(dev)
+    sb = torch.from_numpy(g.integers(115, 135, ((n + 127) // 128, k // 128)).astype(np.uint8)).to(dev)
+    y = torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
+    nbytes = m * k + n * k + m * k / 128 + ((n + 127) // 128) * k / 128 + 2.0 * m * n
+    flops = 2.0 * m * n * k
+    for mode in modes:
+        us = getattr(t, mode)(lambda: fq.block_gemm_ue8m0(tqa, sa, tqb, sb, out=y), reps)
+        emit({"op": "gemm_ue8m0", "M": m, "N": n, "K": k, "mode": mode, "us": us,
+              "TFLOP/s": flops / us / 1e6, "frac_fp8": flops / us / 1e6 / fp8,
+              "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt"], default="all")
+    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt", "gemm_ue8m0"], default="all")
     ap.add_argument("--m", type=int)
     ap.add_argument("--n", type=int)
     ap.add_argument("--k", type=int)
@@ -160,6 +177,8 @@ def main():
         run_gemm(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     elif a.op == "gemm_pt":
         run_gemm_pt(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
+    elif a.op == "gemm_ue8m0":
+        run_gemm_ue8m0(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     else:
         emit({"peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src}})
         for m, _, k in inputs.WORKLOAD_SHAPES[2]:
@@ -171,6 +190,8 @@ def main():
             run_gemm(t, dev, m, n, k, a.reps, modes, hbm, fp8)
         for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
             run_gemm_pt(t, dev, m, n, k, a.reps, modes, hbm, fp8)
+        for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
+            run_gemm_ue8m0(t, dev, m, n, k, a.reps, modes, hbm, fp8)
     if fq.device_status() != 0:
         raise SystemExit("device-side error recorded")
 

@@ -214,6 +214,27 @@ int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa,
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Block-scaled FP8 GEMM with ue8m0 scales (the GEMM of the ue8m0       */
+/* variant above; scales applied by the tensor cores)                   */
+/* ------------------------------------------------------------------ */
+
+/* Y[m,n] = bf16_rne( sum_kb 2^(sa[m,kb]-127) * 2^(sb[n/128,kb]-127)
+ *                     * sum_{k in block kb} A[m,k] * B[n,k] ), fp32 accumulation.
+ *   qa: E4M3 [M,K], row stride lda     sa: E8M0 bytes [M, K/128] contiguous
+ *   qb: E4M3 [N,K], row stride ldb     sb: E8M0 bytes [ceil(N/128), K/128]
+ *   y : bf16 [M,N], row stride ldy
+ * A scale byte of 255 (NaN) makes the outputs it touches NaN.  Shapes,
+ * alignment (none on sa/sb), launch selection, workspace (size from
+ * fp8_block_gemm_workspace_size) and errors as fp8_block_gemm.  The power-of-
+ * two scales multiply the E4M3 products exactly inside the tensor cores
+ * (tcgen05.mma kind::mxf8f6f4.block_scale), so the whole K range
+ * accumulates in TMEM with no per-block promotion. */
+int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa,
+                         const uint8_t* qb, int64_t ldb, const uint8_t* sb,
+                         void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* Block-scaled FP8 GEMM without any allocation                         */
 /* ------------------------------------------------------------------ */
 

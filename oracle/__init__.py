@@ -198,7 +198,8 @@ def e8m0_from_amax(amax: float) -> int:
 def e8m0_to_f32(b) -> np.ndarray:
     """fp32 values 2^(b-127) of E8M0 bytes (NaN for 255)."""
     b = np.asarray(b, dtype=np.uint8)
-    out = np.ldexp(np.ones(b.shape, dtype=np.float64), b.astype(np.int64) - 127).astype(np.float32)
+    e = np.where(b == 255, 0, b.astype(np.int64) - 127)
+    out = np.ldexp(np.ones(b.shape, dtype=np.float64), e).astype(np.float32)
     out[b == 255] = np.nan
     return out
 

@@ -34,6 +34,16 @@ for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 25
     Y = y.float().cpu().numpy().astype(np.float64)
     bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
     assert bad == 0, ("per-tensor", m, n, k, bad)
+    # ue8m0 scales applied by the tensor cores
+    g = np.random.default_rng(m + n)
+    ea = g.integers(115, 135, sa.shape).astype(np.uint8)
+    eb = g.integers(115, 135, sb.shape).astype(np.uint8)
+    y = fq.block_gemm_ue8m0(torch.from_numpy(qa).to(dev), torch.from_numpy(ea).to(dev),
+                            torch.from_numpy(qb).to(dev), torch.from_numpy(eb).to(dev))
+    R, T = oracle.gemm_ue8m0(qa, ea, qb, eb)
+    Y = y.float().cpu().numpy().astype(np.float64)
+    bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
+    assert bad == 0, ("ue8m0", m, n, k, bad)
 assert fq.device_status() == 0
 print("ok")
 '''
