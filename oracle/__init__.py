@@ -71,6 +71,7 @@ def _load():
         lib.oracle_quant_apply.argtypes = [_p, _i64, _i64, _i64, ctypes.c_uint16, _p, _i64, _p]
         lib.oracle_quant_group128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_quant_block128.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
+        lib.oracle_quant_per_channel.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
         lib.oracle_e8m0_from_amax.argtypes = [ctypes.c_float]
         lib.oracle_e8m0_from_amax.restype = ctypes.c_int
         lib.oracle_quant_group128_ue8m0.argtypes = [_p, _i64, _i64, _i64, _p, _i64, _p]
@@ -162,6 +163,15 @@ def quant_apply(x_bits: np.ndarray, amax_bits: int):
     _load().oracle_quant_apply(_ptr(x_bits), m, k, ld, ctypes.c_uint16(int(amax_bits) & 0xFFFF),
                                _ptr(q), k, _ptr(s))
     return q, s[0]
+
+
+def quant_per_channel(x_bits: np.ndarray):
+    """(codes [M,K] uint8, scales [M] float32): one scale per row."""
+    m, k, ld = _rows(x_bits, 2)
+    q = np.empty((m, k), dtype=np.uint8)
+    s = np.empty(m, dtype=np.float32)
+    _load().oracle_quant_per_channel(_ptr(x_bits), m, k, ld, _ptr(q), k, _ptr(s))
+    return q, s
 
 
 def quant_group128(x_bits: np.ndarray):
@@ -275,6 +285,19 @@ def gemm_per_tensor(qa, s_a, qb, s_b):
     sa = np.full((m, k // 128), np.float32(s_a), dtype=np.float32)
     sb = np.full(((n + 127) // 128, k // 128), np.float32(s_b), dtype=np.float32)
     return block_gemm(qa, sa, qb, sb)
+
+
+def gemm_per_channel(qa, sa, qb, sb):
+    """(R, T) of the per-channel-scaled GEMM Y[m,n] = sa[m] * sb[n] * sum_k
+    A[m,k] B[n,k] (one scale per row of A and per row of B): the block GEMM
+    with unit scales gives the exact sums, then one float64 product."""
+    m, k = qa.shape
+    n = qb.shape[0]
+    ones_a = np.ones((m, k // 128), dtype=np.float32)
+    ones_b = np.ones(((n + 127) // 128, k // 128), dtype=np.float32)
+    R, T = block_gemm(qa, ones_a, qb, ones_b)
+    f = np.asarray(sa, np.float64)[:, None] * np.asarray(sb, np.float64)[None, :]
+    return R * f, T * np.abs(f)
 
 
 def gemm_ue8m0(qa, sa_bytes, qb, sb_bytes):

@@ -258,6 +258,21 @@ void oracle_quant_apply(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
             q[r * ldq + c] = quant_one(x[r * ldx + c], s);
 }
 
+/* Per-channel quantisation ([P2] Description names a PER_CHANNEL mode of the
+   same dynamic-quant path and defines nothing more): one scale per row of the
+   matrix -- a token of an activation, an output channel of a weight [N, K] --
+   scale = amax(row) / 448, codes as in the per-tensor path. */
+void oracle_quant_per_channel(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                              uint8_t* q, int64_t ldq, float* scales) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < M; r++) {
+        float s = oracle_scale_from_amax(amax_bf16(x, ldx, r, r + 1, 0, K));
+        scales[r] = s;
+        for (int64_t c = 0; c < K; c++)
+            q[r * ldq + c] = quant_one(x[r * ldx + c], s);
+    }
+}
+
 /* Per-1x128-group quantisation along K ([P1] act_quant with block_size 128):
    for every row m and group g, amax over x[m, 128g : 128g+128], its own
    scale, and codes.  scales is [M, K/128] row-major. */

@@ -541,3 +541,38 @@ def test_gemm_ue8m0_is_integer_matmul_times_powers_of_two(oracle_mod):
         eb = sb[np.arange(300) // 128, kb].astype(np.int64) - 127
         ref += part * np.ldexp(1.0, ea[:, None] + eb[None, :])
     assert np.array_equal(R, ref)
+
+
+# ---------------------------------------------------------------- per-channel
+def test_per_channel_is_per_tensor_of_each_row(oracle_mod):
+    """One scale per row: each row quantised as a one-row tensor."""
+    x = inputs.bf16_bits(inputs.activations_per_tensor(40, k=384))
+    q, s = oracle_mod.quant_per_channel(x)
+    for r in range(40):
+        qr, sr = oracle_mod.quant_per_tensor(np.ascontiguousarray(x[r:r + 1]))
+        assert np.array_equal(q[r], qr[0]) and np.float32(s[r]) == sr
+
+
+def test_per_channel_matches_torch(oracle_mod):
+    x = inputs.activations_per_tensor(64, k=256)
+    xf = x.float()
+    amax = xf.abs().amax(dim=1)
+    s_ref = (amax / 448.0).numpy()
+    q, s = oracle_mod.quant_per_channel(inputs.bf16_bits(x))
+    assert np.array_equal(s.view(np.uint32), s_ref.astype(np.float32).view(np.uint32))
+    ok = s_ref > 0
+    want = torch_encode((xf[ok] / torch.from_numpy(s_ref[ok])[:, None]).numpy())
+    assert np.array_equal(q[ok], want)
+
+
+def test_gemm_per_channel_is_scaled_integer_matmul(oracle_mod):
+    qa, _, qb, _ = inputs.gemm_operands(6, 200, 384, seed=41)
+    g = np.random.default_rng(42)
+    sa = g.uniform(1e-3, 1e-1, 6).astype(np.float32)
+    sb = g.uniform(1e-3, 1e-1, 200).astype(np.float32)
+    R, T = oracle_mod.gemm_per_channel(qa, sa, qb, sb)
+    A = torch_decode(qa)
+    B = torch_decode(qb)
+    f = sa.astype(np.float64)[:, None] * sb.astype(np.float64)[None, :]
+    np.testing.assert_allclose(R, f * (A @ B.T), rtol=1e-12)
+    np.testing.assert_allclose(T, f * (np.abs(A) @ np.abs(B).T), rtol=1e-12)
