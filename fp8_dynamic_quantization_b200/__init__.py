@@ -25,7 +25,8 @@ from . import _abi
 __all__ = [
     "act_quant_per_tensor", "act_amax", "act_quant_apply", "act_quant_group128",
     "weight_quant_block128", "act_quant_group128_ue8m0", "weight_quant_block128_ue8m0",
-    "block_gemm_ue8m0", "linear_ue8m0",
+    "block_gemm_ue8m0", "linear_ue8m0", "act_quant_per_channel", "gemm_per_channel",
+    "linear_per_channel",
     "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
     "device_status",
     "per_tensor_sharded", "Fp8qError", "library",
@@ -145,6 +146,21 @@ def weight_quant_block128(w: torch.Tensor):
     return q.view(E4M3), s
 
 
+def act_quant_per_channel(x: torch.Tensor):
+    """Per-channel (per-row) quantisation of bf16 x[M,K] (K % 8 == 0).
+
+    Returns (codes [M,K] float8_e4m3fn, scales [M] float32)."""
+    lib = _abi.load()
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    M, K, ldx = _rows(x, "x")
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s = torch.empty(M, dtype=torch.float32, device=x.device)
+    _abi.check(lib.fp8_act_quant_per_channel(x.data_ptr(), M, K, ldx, q.data_ptr(), K, s.data_ptr(),
+                                             _stream(x.device)), "fp8_act_quant_per_channel")
+    return q.view(E4M3), s
+
+
 def act_quant_group128_ue8m0(x: torch.Tensor):
     """Per-1x128-group quantisation with power-of-two (ue8m0) scales.
 
@@ -244,6 +260,42 @@ def linear_per_tensor(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> to
     weight codes qb with scale sb."""
     qa, sa = act_quant_per_tensor(x)
     return gemm_per_tensor(qa, sa, qb, sb)
+
+
+def gemm_per_channel(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                     out: torch.Tensor | None = None) -> torch.Tensor:
+    """bf16 Y[M,N] = sa[m] * sb[n] * A * B^T with one fp32 scale per row of A
+    (sa [M]) and per row of B (sb [N], an output channel)."""
+    lib = _abi.load()
+    M, K, lda = _rows(_codes(qa, "qa"), "qa")
+    N, Kb, ldb = _rows(_codes(qb, "qb"), "qb")
+    if K != Kb:
+        raise ValueError("qa and qb must share K")
+    if sa.dtype != torch.float32 or tuple(sa.shape) != (M,) or not sa.is_contiguous():
+        raise ValueError("sa must be a contiguous float32 [M] tensor")
+    if sb.dtype != torch.float32 or tuple(sb.shape) != (N,) or not sb.is_contiguous():
+        raise ValueError("sb must be a contiguous float32 [N] tensor")
+    if out is None:
+        ldy_alloc = (N + 7) // 8 * 8
+        out = torch.empty((M, ldy_alloc), dtype=torch.bfloat16, device=qa.device)[:, :N]
+    _, _, ldy = _rows(out, "out")
+    nbytes = lib.fp8_block_gemm_workspace_size(M, N, K)
+    ws_ptr, ws_len = None, 0
+    if nbytes:
+        ws = _workspace("gemm", qa.device, nbytes, zero=False)
+        ws_ptr, ws_len = ws.data_ptr(), ws.numel()
+    _abi.check(lib.fp8_gemm_per_channel(qa.data_ptr(), lda, sa.data_ptr(), qb.data_ptr(), ldb, sb.data_ptr(),
+                                        out.data_ptr(), ldy, M, N, K, ws_ptr, ws_len, _stream(qa.device)),
+               "fp8_gemm_per_channel")
+    return out
+
+
+def linear_per_channel(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:
+    """The dynamic FP8 linear method with per-channel scales: per-token
+    quantisation of x, then the GEMM against weight codes qb with one scale
+    per output channel (sb [N])."""
+    qa, sa = act_quant_per_channel(x)
+    return gemm_per_channel(qa, sa, qb, sb)
 
 
 def block_gemm_ue8m0(qa: torch.Tensor, sa: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,

@@ -98,6 +98,13 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 2>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 2>();
                 if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, 2>();
@@ -570,6 +577,24 @@ int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw, 
     return run_block128(w, N, K, ldw, qb, ldqb, sb, false, stream);
 }
 
+int fp8_act_quant_per_channel(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
+                              int64_t ldq, float* scales, void* stream) {
+    int rc = check_bf16_matrix(x, M, K, ldx, q, ldq, 8);
+    if (rc != FP8Q_OK) return rc;
+    if (M == 0) return FP8Q_OK;
+    if (!scales) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned4(scales)) return FP8Q_ERR_MISALIGNED;
+    DeviceInfo* d = nullptr;
+    if ((rc = device_info(&d)) != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int grid = int(std::max<int64_t>(1, std::min<int64_t>(M, int64_t(d->sms) * kBlocksPerSm)));
+    if (log_enabled())
+        std::fprintf(stderr, "[fp8q] per_channel M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
+    per_channel_quant_kernel<<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x), M, K / 8, ldx,
+                                                            q, ldq, scales);
+    return launch_status();
+}
+
 int fp8_act_quant_group128_ue8m0(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_t* q,
                                  int64_t ldq, uint8_t* scales, void* stream) {
     return run_group128(x, M, K, ldx, q, ldq, scales, true, stream);
@@ -593,8 +618,9 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                     void* workspace, size_t workspace_bytes, void* stream, int mode) {
-    // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes
-    const bool per_tensor = mode == 1, ue8m0 = mode == 2;
+    // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes;
+    // 3: per-channel fp32 scales
+    const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
@@ -655,7 +681,22 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
-    if (ue8m0) {
+    if (per_channel) {
+        if (pl.swap) {
+            switch (pl.bn) {
+                case 16: launch_gemm<16, true, 12, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 32: launch_gemm<32, true, 10, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                case 64: launch_gemm<64, true, 8, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+                default: launch_gemm<128, true, 6, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
+            }
+        } else if (pl.bn == 128) {
+            launch_gemm<128, false, 6, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else if (pl.bn == 192) {
+            launch_gemm<192, false, 5, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else {
+            launch_gemm<256, false, 4, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+        }
+    } else if (ue8m0) {
         if (pl.swap) {
             switch (pl.bn) {
                 case 16: launch_gemm<16, true, 12, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st); break;
@@ -724,6 +765,12 @@ int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa, const u
                         const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream) {
     return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 1);
+}
+
+int fp8_gemm_per_channel(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
+                         const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream) {
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 3);
 }
 
 int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa, const uint8_t* qb, int64_t ldb,

@@ -53,6 +53,9 @@
 //      block-scaled MMA reads: A row m at lane m, column base + m/32; B row n
 //      at column base + n/32 in every lane quarter; the byte picked by the
 //      instruction's scale-factor id, here kb % 4.
+//   3  per-channel scales (sa [M] per row of A, sb [N] per row of B): one
+//      TMEM accumulation per unit; the epilogue multiplies row m by its
+//      scale and column n by the one staged for the tile in shared memory.
 #pragma once
 
 #include <cuda.h>
@@ -78,6 +81,7 @@ template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS 
 struct GemmCfg {
     static constexpr bool PT = SM == 1;                        // per-tensor scales
     static constexpr bool MX = SM == 2;                        // ue8m0 scales applied by the MMA
+    static constexpr bool PC = SM == 3;                        // per-channel scales
     // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
     // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
     // and its TMEM receives its 128 rows x BN columns of every product.
@@ -107,7 +111,8 @@ struct GemmCfg {
     static constexpr int kTmemCols = MX ? 512 : kNumBuf * BN <= 32 ? 32 : kNumBuf * BN <= 64 ? 64
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
     static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
-    static constexpr int kSlabFloats = (SWAP && SM == 0) ? BN * kMaxUnitKb : 0;  // swapped-mode scale slab
+    // swapped-mode scale slab (block scales); per-channel: the tile's column scales
+    static constexpr int kSlabFloats = (SWAP && SM == 0) ? BN * kMaxUnitKb : PC ? BN : 0;
     // SS: block scales staged through shared memory.  The producer copies,
     // per group of 4 K blocks, the tile's 128 x 4 row scales and its
     // BN/128 x 4 column-block scales into a ring of kScaleSlots slots.
@@ -236,8 +241,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmSB,    // column-block scales [NB, G] fp32 (SS only)
                   const GemmParams p) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
-    constexpr bool PT = C::PT, MX = C::MX;
-    constexpr bool ONE = PT || MX;        // one TMEM accumulation per unit, no per-K-block promotion
+    constexpr bool PT = C::PT, MX = C::MX, PC = C::PC;
+    constexpr bool ONE = PT || MX || PC;  // one TMEM accumulation per unit, no per-K-block promotion
     constexpr int NB = C::kNumBuf;
     constexpr uint32_t kSlots = C::kScaleSlots > 0 ? C::kScaleSlots : 1;   // divisor for the (SS) slot ring
     constexpr uint32_t kSfN = C::kSfSlots > 0 ? C::kSfSlots : 1;         // divisor for the (MX) slot ring
@@ -485,6 +490,15 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             const int q0 = tq * BN;
             const int m_row = tp * C::kTileRows + int(rank) * 128 + row;   // normal: token row
             const int n_row = tp * 128 + row;                              // swapped: weight row
+            if (PC) {
+                // slab[j] = scale of tile column j: sb[q0+j] (normal) or sa[q0+j] (swapped)
+                ptx::named_bar_sync(1, nthreads);
+                for (int i = etid; i < BN; i += nthreads) {
+                    const int qi = q0 + i;
+                    slab[i] = SWAP ? (qi < p.M ? __ldg(p.sa + qi) : 0.0f) : (qi < p.N ? __ldg(p.sb + qi) : 0.0f);
+                }
+                ptx::named_bar_sync(1, nthreads);
+            }
             if (SWAP && SM == 0) {
                 // slab[kbl*BN + j] = sa[q0+j, kb0+kbl] * sb[tp, kb0+kbl]
                 ptx::named_bar_sync(1, nthreads);
@@ -518,7 +532,12 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             bool ok = true;
             // per-tensor scales: one step per unit, one scalar scale
             const int kb_last = ONE ? kb0 + 1 : kb1;
-            const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : MX ? 1.0f : 0.0f;
+            // one-step modes: the scale applied to the whole accumulation
+            // (per-channel: this thread's row; its column scales come later)
+            const float s_pt = PT ? __ldg(p.sa) * __ldg(p.sb) : MX ? 1.0f
+                             : PC ? (SWAP ? (n_row < p.N ? __ldg(p.sb + n_row) : 0.0f)
+                                          : (m_row < p.M ? __ldg(p.sa + m_row) : 0.0f))
+                             : 0.0f;
             for (int kb = kb0; kb < kb_last; ++kb, ++c) {
                 float s = s_pt;
                 if (SS) {
@@ -581,6 +600,10 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
             float acc[C::kCW];
 #pragma unroll
             for (int j = 0; j < C::kCW / 2; ++j) ptx::unpack_f32x2(acc2[j], acc[2 * j], acc[2 * j + 1]);
+            if (PC) {
+#pragma unroll
+                for (int j = 0; j < C::kCW; ++j) acc[j] *= slab[chalf * C::kCW + j];
+            }
             if (p.splits == 1) {
                 if (!SWAP) {
                     const int m = m_row;

@@ -19,6 +19,8 @@
 //  per_tensor_cluster_kernel small tensors: one launch of one thread-block
 //                            cluster; values stay in registers while the
 //                            CTAs exchange partial maxima on chip.
+//  per_channel_quant_kernel  one scale per row (a token, or an output
+//                            channel of a weight).
 //  block128_quant_kernel     128x128 weight blocks (offline step).
 //  Both group and block kernels also have a ue8m0 form (E8 = true): the
 //  scale is the smallest power of two >= amax/448, written as an E8M0 byte.
@@ -261,6 +263,38 @@ reduce_partials_kernel(const uint32_t* __restrict__ partials, int n, uint32_t* _
 // scale = amax / 448 from an amax word, for an empty apply.
 __global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float* __restrict__ scale) {
     if (threadIdx.x == 0) *scale = scale_from_amax_bits(*amax_bits & 0x7FFFu);
+}
+
+// ---------------------------------------------------------------------------
+// Per-channel (per-row) quantisation: one CTA per row at a time.  Pass 1
+// reduces the row's amax with 16-byte loads; pass 2 re-reads the row, which
+// is still in L2 (at most a few thousand rows are in flight), and writes
+// the codes.  vpr = 16-byte vectors per row.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQuantThreads)
+per_channel_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t vpr, int64_t ldx,
+                         uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scales) {
+    __shared__ uint32_t red[kQuantThreads / 32];
+    for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
+        const uint16_t* xr = x + r * ldx;
+        uint32_t m = 0;
+        for (int64_t i = threadIdx.x; i < vpr; i += 4 * kQuantThreads) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int64_t j = i + u * kQuantThreads;
+                v[u] = j < vpr ? ld_stream16(xr + j * 8) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m = max(m, absmax8(v[u]));
+        }
+        m = block_max<kQuantThreads>(m, red);
+        const Scale d = make_scale(scale_from_amax_bits(m));
+        if (threadIdx.x == 0) scales[r] = d.s;
+        uint8_t* qr = q + r * ldq;
+        for (int64_t i = threadIdx.x; i < vpr; i += kQuantThreads)
+            st_stream8(qr + i * 8, quant8(ld_stream16(xr + i * 8), d));
+    }
 }
 
 // ---------------------------------------------------------------------------

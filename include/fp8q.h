@@ -147,6 +147,31 @@ int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw,
                               uint8_t* qb, int64_t ldqb, float* sb, void* stream);
 
 /* ------------------------------------------------------------------ */
+/* Per-channel scales ([P2] Description names a PER_CHANNEL mode of the */
+/* dynamic-quant path and defines nothing more).  Reading: one fp32      */
+/* scale per row of the quantised matrix -- a token of X, an output     */
+/* channel of a weight W[N,K] -- scale = amax(row)/448, codes as in the */
+/* per-tensor path (zero row: scale 0, signed-zero codes).              */
+/* ------------------------------------------------------------------ */
+
+/* x: bf16 [M,K] (row stride ldx, K a multiple of 8).  Writes q: uint8
+ * [M,K] (row stride ldq) and scales: fp32 [M].  No workspace. */
+int fp8_act_quant_per_channel(const void* x, int64_t M, int64_t K, int64_t ldx,
+                              uint8_t* q, int64_t ldq, float* scales, void* stream);
+
+/* Y[m,n] = bf16_rne( sa[m] * sb[n] * sum_k A[m,k] * B[n,k] ), fp32
+ * accumulation of the sum in TMEM, the two scales applied in the epilogue.
+ *   qa: E4M3 [M,K] (row stride lda), sa: fp32 [M] on the device
+ *   qb: E4M3 [N,K] (row stride ldb), sb: fp32 [N] on the device
+ *   y : bf16 [M,N] (row stride ldy)
+ * Shapes, alignment, launch selection, workspace and errors as
+ * fp8_block_gemm. */
+int fp8_gemm_per_channel(const uint8_t* qa, int64_t lda, const float* sa,
+                         const uint8_t* qb, int64_t ldb, const float* sb,
+                         void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------------ */
 /* ue8m0 (power-of-two) scales ([P1] Benchmarking the Activation        */
 /* Quantization Kernel: act_quant(..., scale_fmt="ue8m0")).  The page   */
 /* names the format only.  Reading: the scale is the smallest power of  */

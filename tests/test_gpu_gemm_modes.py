@@ -44,6 +44,15 @@ for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 25
     Y = y.float().cpu().numpy().astype(np.float64)
     bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
     assert bad == 0, ("ue8m0", m, n, k, bad)
+    # per-channel scales applied in the epilogue
+    ra = g.uniform(1e-3, 1e-1, m).astype(np.float32)
+    rb = g.uniform(1e-3, 1e-1, n).astype(np.float32)
+    y = fq.gemm_per_channel(torch.from_numpy(qa).to(dev), torch.from_numpy(ra).to(dev),
+                            torch.from_numpy(qb).to(dev), torch.from_numpy(rb).to(dev))
+    R, T = oracle.gemm_per_channel(qa, ra, qb, rb)
+    Y = y.float().cpu().numpy().astype(np.float64)
+    bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
+    assert bad == 0, ("per-channel", m, n, k, bad)
 assert fq.device_status() == 0
 print("ok")
 '''
