@@ -590,7 +590,7 @@ int fp8_act_quant_per_channel(const void* x, int64_t M, int64_t K, int64_t ldx, 
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(M, int64_t(d->sms) * kBlocksPerSm)));
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] per_channel M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
-    per_channel_quant_kernel<<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x), M, K / 8, ldx,
+    per_channel_quant_kernel<4><<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x), M, K / 8, ldx,
                                                             q, ldq, scales);
     return launch_status();
 }

@@ -266,15 +266,47 @@ __global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float*
 }
 
 // ---------------------------------------------------------------------------
-// Per-channel (per-row) quantisation: one CTA per row at a time.  Pass 1
-// reduces the row's amax with 16-byte loads; pass 2 re-reads the row, which
-// is still in L2 (at most a few thousand rows are in flight), and writes
-// the codes.  vpr = 16-byte vectors per row.
+// Per-channel (per-row) quantisation: one CTA per row at a time.  A row of
+// up to U*256*8 values stays in registers (one read of x); the CTA loads its
+// next row before reducing the current one, so the loads of one row overlap
+// the reduction and stores of the previous.  Longer rows take two passes,
+// the second re-reading the row from L2 (at most a few thousand rows are in
+// flight).  vpr = 16-byte vectors per row.
 // ---------------------------------------------------------------------------
+template <int U>
 __global__ void __launch_bounds__(kQuantThreads)
 per_channel_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t vpr, int64_t ldx,
                          uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scales) {
     __shared__ uint32_t red[kQuantThreads / 32];
+    if (vpr <= int64_t(U) * kQuantThreads) {
+        uint4 cur[U], nxt[U];
+        auto load = [&](int64_t r, uint4* v) {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t j = threadIdx.x + int64_t(u) * kQuantThreads;
+                v[u] = (r < M && j < vpr) ? ld_stream16(x + r * ldx + j * 8) : make_uint4(0, 0, 0, 0);
+            }
+        };
+        int64_t r = blockIdx.x;
+        load(r, cur);
+        for (; r < M; r += gridDim.x) {
+            load(r + gridDim.x, nxt);
+            uint32_t m = 0;
+#pragma unroll
+            for (int u = 0; u < U; ++u) m = max(m, absmax8(cur[u]));
+            m = block_max<kQuantThreads>(m, red);
+            const Scale d = make_scale(scale_from_amax_bits(m));
+            if (threadIdx.x == 0) scales[r] = d.s;
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int64_t j = threadIdx.x + int64_t(u) * kQuantThreads;
+                if (j < vpr) st_stream8(q + r * ldq + j * 8, quant8(cur[u], d));
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+        }
+        return;
+    }
     for (int64_t r = blockIdx.x; r < M; r += gridDim.x) {
         const uint16_t* xr = x + r * ldx;
         uint32_t m = 0;

@@ -106,6 +106,41 @@ def run_group(t, dev, m, k, reps, modes, hbm):
               "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
 
 
+def run_per_channel(t, dev, m, k, reps, modes, hbm):
+    x = inputs.activations_per_tensor(m, k=k).to(dev)
+    nbytes = 3.0 * m * k + 4.0 * m
+    for mode in modes:
+        us = getattr(t, mode)(lambda: fq.act_quant_per_channel(x), reps)
+        emit({"op": "per_channel_quant", "M": m, "K": k, "mode": mode, "us": us,
+              "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
+def run_group_ue8m0(t, dev, m, k, reps, modes, hbm):
+    x = inputs.activations_group(m, k=k).to(dev)
+    nbytes = 3.0 * m * k + m * (k // 128)
+    for mode in modes:
+        us = getattr(t, mode)(lambda: fq.act_quant_group128_ue8m0(x), reps)
+        emit({"op": "group128_quant_ue8m0", "M": m, "K": k, "mode": mode, "us": us,
+              "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
+def run_gemm_pc(t, dev, m, n, k, reps, modes, hbm, fp8):
+    qa, _, qb, _ = inputs.gemm_operands(m, n, k)
+    g = np.random.default_rng(m + n)
+    tqa = torch.from_numpy(qa).to(dev).view(torch.float8_e4m3fn)
+    tqb = torch.from_numpy(qb).to(dev).view(torch.float8_e4m3fn)
+    sa = torch.from_numpy(g.uniform(1e-3, 1e-1, m).astype(np.float32)).to(dev)
+    sb = torch.from_numpy(g.uniform(1e-3, 1e-1, n).astype(np.float32)).to(dev)
+    y = torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
+    nbytes = m * k + n * k + 4.0 * (m + n) + 2.0 * m * n
+    flops = 2.0 * m * n * k
+    for mode in modes:
+        us = getattr(t, mode)(lambda: fq.gemm_per_channel(tqa, sa, tqb, sb, out=y), reps)
+        emit({"op": "gemm_per_channel", "M": m, "N": n, "K": k, "mode": mode, "us": us,
+              "TFLOP/s": flops / us / 1e6, "frac_fp8": flops / us / 1e6 / fp8,
+              "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
 def run_gemm(t, dev, m, n, k, reps, modes, hbm, fp8):
     qa, sa, qb, sb = inputs.gemm_operands(m, n, k)
     tqa = torch.from_numpy(qa).to(dev).view(torch.float8_e4m3fn)
@@ -157,7 +192,8 @@ def run_gemm_ue8m0(t, dev, m, n, k, reps, modes, hbm, fp8):
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt", "gemm_ue8m0"], default="all")
+    ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt", "gemm_ue8m0",
+                                     "per_channel", "group128_ue8m0", "gemm_pc"], default="all")
     ap.add_argument("--m", type=int)
     ap.add_argument("--n", type=int)
     ap.add_argument("--k", type=int)
@@ -179,6 +215,12 @@ def main():
         run_gemm_pt(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     elif a.op == "gemm_ue8m0":
         run_gemm_ue8m0(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
+    elif a.op == "per_channel":
+        run_per_channel(t, dev, a.m, a.k or 7168, a.reps, modes, hbm)
+    elif a.op == "group128_ue8m0":
+        run_group_ue8m0(t, dev, a.m, a.k or 7168, a.reps, modes, hbm)
+    elif a.op == "gemm_pc":
+        run_gemm_pc(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     else:
         emit({"peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src}})
         for m, _, k in inputs.WORKLOAD_SHAPES[2]:
@@ -192,6 +234,11 @@ def main():
             run_gemm_pt(t, dev, m, n, k, a.reps, modes, hbm, fp8)
         for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
             run_gemm_ue8m0(t, dev, m, n, k, a.reps, modes, hbm, fp8)
+        for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
+            run_gemm_pc(t, dev, m, n, k, a.reps, modes, hbm, fp8)
+        for m, _, k in inputs.WORKLOAD_SHAPES[3]:
+            run_group_ue8m0(t, dev, m, k, a.reps, modes, hbm)
+            run_per_channel(t, dev, m, k, a.reps, modes, hbm)
     if fq.device_status() != 0:
         raise SystemExit("device-side error recorded")
 
