@@ -27,7 +27,7 @@ __all__ = [
     "weight_quant_block128", "act_quant_group128_ue8m0", "weight_quant_block128_ue8m0",
     "block_gemm_ue8m0", "linear_ue8m0", "act_quant_per_channel", "gemm_per_channel",
     "linear_per_channel",
-    "block_gemm", "linear", "gemm_per_tensor", "linear_per_tensor",
+    "block_gemm", "linear", "linear_fused", "gemm_per_tensor", "linear_per_tensor",
     "device_status",
     "per_tensor_sharded", "Fp8qError", "library",
 ]
@@ -332,6 +332,34 @@ def linear_ue8m0(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.T
     qb with E8M0 block scales sb."""
     qa, sa = act_quant_group128_ue8m0(x)
     return block_gemm_ue8m0(qa, sa, qb, sb)
+
+
+def linear_fused(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """linear() in one call, bit-identical to act_quant_group128 followed by
+    block_gemm: the GEMM is launched as a programmatic dependent of the
+    quantisation, so its weight loads start while the tokens are quantised."""
+    lib = _abi.load()
+    if x.dtype != torch.bfloat16:
+        raise TypeError("x must be bfloat16")
+    M, K, ldx = _rows(x, "x")
+    N, Kb, ldb = _rows(_codes(qb, "qb"), "qb")
+    if K != Kb:
+        raise ValueError("x and qb must share K")
+    if sb.dtype != torch.float32 or tuple(sb.shape) != ((N + 127) // 128, K // 128) or not sb.is_contiguous():
+        raise ValueError("sb must be a contiguous float32 [ceil(N/128), K/128] tensor")
+    if out is None:
+        ldy_alloc = (N + 7) // 8 * 8
+        out = torch.empty((M, ldy_alloc), dtype=torch.bfloat16, device=x.device)[:, :N]
+    _, _, ldy = _rows(out, "out")
+    nbytes = lib.fp8_linear_group128_workspace_size(M, N, K)
+    ws_ptr, ws_len = None, 0
+    if nbytes:
+        ws = _workspace("linear", x.device, nbytes, zero=False)
+        ws_ptr, ws_len = ws.data_ptr(), ws.numel()
+    _abi.check(lib.fp8_linear_group128(x.data_ptr(), ldx, qb.data_ptr(), ldb, sb.data_ptr(), out.data_ptr(), ldy,
+                                       M, N, K, ws_ptr, ws_len, _stream(x.device)), "fp8_linear_group128")
+    return out
 
 
 def linear(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:

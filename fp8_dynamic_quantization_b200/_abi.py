@@ -29,6 +29,8 @@ SIGNATURES = {
     "fp8_act_quant_apply": (_int, [_p, _i64, _i64, _i64, _p, _p, _i64, _p, _p]),
     "fp8_act_quant_group128": (_int, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),
     "fp8_weight_quant_block128": (_int, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),
+    "fp8_linear_group128_workspace_size": (_sz, [_i64, _i64, _i64]),
+    "fp8_linear_group128": (_int, [_p, _i64, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8_act_quant_per_channel": (_int, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),
     "fp8_gemm_per_channel": (_int, [_p, _i64, _p, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8_act_quant_group128_ue8m0": (_int, [_p, _i64, _i64, _i64, _p, _i64, _p, _p]),

@@ -98,6 +98,8 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<16, true, 8, false, 4>();
+                if (e == cudaSuccess) e = set_gemm_smem<32, true, 7, false, 4>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, 3>();
@@ -305,11 +307,42 @@ bool make_scale_tmap(CUtensorMap* m, const float* base, int64_t rows, int64_t G,
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Map of bf16 tokens x [rows, K] (row pitch ldx elements, a multiple of 8):
+// boxes of one 128-wide K block x box_rows rows, no swizzle; rows past the
+// end read as zero.
+bool make_x_tmap(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t K, int64_t ldx, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(ldx) * 2};
+    cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // tsa/tsb: scale maps (staged-scale variants only; the others ignore them)
 template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& tsa, const CUtensorMap& tsb,
                  const GemmParams& p, int grid, cudaStream_t st) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
+    if (!PAIR && p.pdl) {
+        // programmatic dependent launch: may start while the previous kernel
+        // in the stream runs; the kernel waits for it before reading A or sa
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(unsigned(grid));
+        cfg.blockDim = dim3(C::kThreads);
+        cfg.dynamicSmemBytes = C::kSmemBytes;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, tp, tq, tsa, tsb, p);
+        return;
+    }
     if (!PAIR) {
         block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS><<<grid, C::kThreads, C::kSmemBytes, st>>>(
             tp, tq, tsa, tsb, p);
@@ -617,18 +650,22 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                    void* workspace, size_t workspace_bytes, void* stream, int mode) {
+                    void* workspace, size_t workspace_bytes, void* stream, int mode,
+                    const uint16_t* x = nullptr, int64_t ldx = 0, bool pdl = false) {
     // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes;
-    // 3: per-channel fp32 scales
-    const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3;
+    // 3: per-channel fp32 scales; 4: fp32 block scales with the group-128
+    // quantisation of bf16 tokens x fused in (swapped tiles of <= 64 tokens;
+    // qa and sa unused)
+    const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3, fused = mode == 4;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 || N == 0) return FP8Q_OK;
-    if (!qa || !sa || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
-    if (lda < K || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
-    if (!aligned16(qa) || !aligned16(qb) || !aligned16(y) || lda % 16 || ldb % 16 || (ldy * 2) % 16 ||
-        (!ue8m0 && (!aligned4(sa) || !aligned4(sb))))
+    if ((fused ? !x : (!qa || !sa)) || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+    if ((fused ? ldx < K : lda < K) || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+    if ((fused ? (!aligned16(x) || ldx % 8) : (!aligned16(qa) || lda % 16)) ||
+        !aligned16(qb) || !aligned16(y) || ldb % 16 || (ldy * 2) % 16 ||
+        (!ue8m0 && ((!fused && !aligned4(sa)) || !aligned4(sb))))
         return FP8Q_ERR_MISALIGNED;
     DeviceInfo* d = nullptr;
     int rc = device_info(&d);
@@ -649,9 +686,10 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     const uint8_t* Q = pl.swap ? qa : qb;
     const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
     const int64_t ld_p = pl.swap ? ldb : lda, ld_q = pl.swap ? lda : ldb;
-    if (!make_tmap(&tp, P, rows_p, K, ld_p, 128) ||
-        !make_tmap(&tq, Q, rows_q, K, ld_q, pl.pair ? pl.bn / 2 : pl.bn))
-        return FP8Q_ERR_CUDA;
+    if (fused && !(pl.swap && pl.bn <= 32)) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (!make_tmap(&tp, P, rows_p, K, ld_p, 128)) return FP8Q_ERR_CUDA;
+    if (fused) tq = tp;                            // the token operand is written by the kernel
+    else if (!make_tmap(&tq, Q, rows_q, K, ld_q, pl.pair ? pl.bn / 2 : pl.bn)) return FP8Q_ERR_CUDA;
     GemmParams p;
     p.sa = sa;
     p.sb = sb;
@@ -668,6 +706,9 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     p.units = pl.units;
     p.scale_vec4 = mode == 0 && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
     p.sf_words = ue8m0 && (p.G % 4 == 0) && aligned4(sa) && aligned4(sb);
+    p.x = x;
+    p.ldx = ldx;
+    p.pdl = (pdl && mode == 0 && !pl.pair) ? 1 : 0;
     // Normal 128/256-wide tiles stage the block scales through shared memory
     // (TMA boxes of 4 K blocks) when the scale rows allow 16-byte boxes.
     const bool staged = p.scale_vec4 && !pl.swap && !pl.pair && (pl.bn == 128 || pl.bn == 256);
@@ -675,13 +716,17 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     if (staged && (!make_scale_tmap(&tsa, sa, M, p.G, 128) ||
                    !make_scale_tmap(&tsb, sb, (N + 127) / 128, p.G, pl.bn / 128)))
         return FP8Q_ERR_CUDA;
+    if (fused && !make_x_tmap(&tsa, x, M, K, ldx, pl.bn)) return FP8Q_ERR_CUDA;   // the token tiles
     p.wait_budget = wait_budget_cycles();
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d\n",
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid);
-    if (per_channel) {
+    if (fused) {
+        if (pl.bn == 16) launch_gemm<16, true, 8, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
+        else launch_gemm<32, true, 7, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
+    } else if (per_channel) {
         if (pl.swap) {
             switch (pl.bn) {
                 case 16: launch_gemm<16, true, 12, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
@@ -765,6 +810,61 @@ int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa, const u
                         const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream) {
     return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 1);
+}
+
+// ------------------------------------------------------------ fused linear
+// FP8Q_LINEAR selects how fp8_linear_group128 runs (measurement only; every
+// choice computes the same bytes): unset -> quantisation kernel, then the
+// GEMM as a programmatic dependent; "fused" -> quantisation inside the GEMM
+// for swapped tiles of <= 32 tokens; "serial" -> the two kernels without
+// launch overlap.
+static const char* linear_mode() {
+    static const char* v = [] { const char* e = std::getenv("FP8Q_LINEAR"); return e ? e : ""; }();
+    return v;
+}
+static bool linear_in_kernel_quant() { return std::strcmp(linear_mode(), "fused") == 0; }
+static bool linear_without_overlap() { return std::strcmp(linear_mode(), "serial") == 0; }
+
+// Workspace layout when the launch is not fused: codes [M, K], then the
+// group scales [M, K/128] fp32, then the GEMM's split-K partials.
+static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
+
+size_t fp8_linear_group128_workspace_size(int64_t M, int64_t N, int64_t K) {
+    if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
+    DeviceInfo* d = nullptr;
+    if (device_info(&d) != FP8Q_OK) return 0;
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms);
+    if (linear_in_kernel_quant() && pl.swap && pl.bn <= 32) return pl.ws_bytes;
+    return round256(size_t(M) * size_t(K)) + round256(size_t(M) * size_t(K / 128) * 4) + pl.ws_bytes;
+}
+
+int fp8_linear_group128(const void* x, int64_t ldx, const uint8_t* qb, int64_t ldb, const float* sb,
+                        void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
+    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return FP8Q_OK;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc != FP8Q_OK) return rc;
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms);
+    if (linear_in_kernel_quant() && pl.swap && pl.bn <= 32) {
+        if (log_enabled())
+            std::fprintf(stderr, "[fp8q] linear M=%lld N=%lld K=%lld: group-128 quantisation fused into the GEMM\n",
+                         (long long)M, (long long)N, (long long)K);
+        return run_gemm(nullptr, 0, nullptr, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 4,
+                        static_cast<const uint16_t*>(x), ldx);
+    }
+    const size_t need = fp8_linear_group128_workspace_size(M, N, K);
+    if (!workspace || workspace_bytes < need) return FP8Q_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
+    uint8_t* qa = static_cast<uint8_t*>(workspace);
+    float* sa = reinterpret_cast<float*>(qa + round256(size_t(M) * size_t(K)));
+    uint8_t* gws = reinterpret_cast<uint8_t*>(sa) + round256(size_t(M) * size_t(K / 128) * 4);
+    if ((rc = run_group128(x, M, K, ldx, qa, K, sa, false, stream)) != FP8Q_OK) return rc;
+    // the GEMM starts its weight loads while the quantisation runs
+    return run_gemm(qa, K, sa, qb, ldb, sb, y, ldy, M, N, K, gws, pl.ws_bytes, stream, 0,
+                    nullptr, 0, !linear_without_overlap());
 }
 
 int fp8_gemm_per_channel(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,

@@ -228,6 +228,11 @@ __host__ __device__ constexpr uint32_t idesc_mx_e4m3(int n, uint32_t sf_id) {
          | (sf_id << 29);                  // A scale-factor id
 }
 
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their memory is visible; let dependents start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Make this thread's generic-proxy shared-memory writes visible to the
 // async proxy (tcgen05.cp, TMA) before it signals them.
 __device__ __forceinline__ void fence_proxy_async_shared() {

@@ -56,6 +56,8 @@ __global__ void __launch_bounds__(kQuantThreads)
 group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                       uint8_t* __restrict__ q, int64_t ldq,
                       void* __restrict__ scales, int64_t groups, int64_t G) {
+    // a GEMM launched as a programmatic dependent may start its weight loads now
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int sub = threadIdx.x & 7;
     const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 3;
     const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 3;

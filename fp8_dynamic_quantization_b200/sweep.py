@@ -141,6 +141,27 @@ def run_gemm_pc(t, dev, m, n, k, reps, modes, hbm, fp8):
               "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
 
 
+def run_linear(t, dev, m, n, k, reps, modes, hbm, fp8):
+    """The group-128 linear two ways: quantisation fused into the GEMM, and
+    act_quant_group128 followed by block_gemm."""
+    x = inputs.activations_group(m, k=k).to(dev)
+    qb, sb = inputs.weight_operands(n, k)
+    tqb = torch.from_numpy(qb).to(dev).view(torch.float8_e4m3fn)
+    tsb = torch.from_numpy(sb).to(dev)
+    y = torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
+    nbytes = 2.0 * m * k + n * k + 4.0 * ((n + 127) // 128) * (k // 128) + 2.0 * m * n
+    flops = 2.0 * m * n * k
+
+    def two_step():
+        qa, sa = fq.act_quant_group128(x)
+        fq.block_gemm(qa, sa, tqb, tsb, out=y)
+    for mode in modes:
+        for name, fn in (("linear_fused", lambda: fq.linear_fused(x, tqb, tsb, out=y)), ("linear_two_step", two_step)):
+            us = getattr(t, mode)(fn, reps)
+            emit({"op": name, "M": m, "N": n, "K": k, "mode": mode, "us": us,
+                  "TFLOP/s": flops / us / 1e6, "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm})
+
+
 def run_gemm(t, dev, m, n, k, reps, modes, hbm, fp8):
     qa, sa, qb, sb = inputs.gemm_operands(m, n, k)
     tqa = torch.from_numpy(qa).to(dev).view(torch.float8_e4m3fn)
@@ -193,7 +214,7 @@ def run_gemm_ue8m0(t, dev, m, n, k, reps, modes, hbm, fp8):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--op", choices=["all", "per_tensor", "group128", "gemm", "gemm_pt", "gemm_ue8m0",
-                                     "per_channel", "group128_ue8m0", "gemm_pc"], default="all")
+                                     "per_channel", "group128_ue8m0", "gemm_pc", "linear"], default="all")
     ap.add_argument("--m", type=int)
     ap.add_argument("--n", type=int)
     ap.add_argument("--k", type=int)
@@ -221,6 +242,8 @@ def main():
         run_group_ue8m0(t, dev, a.m, a.k or 7168, a.reps, modes, hbm)
     elif a.op == "gemm_pc":
         run_gemm_pc(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
+    elif a.op == "linear":
+        run_linear(t, dev, a.m, a.n, a.k or 7168, a.reps, modes, hbm, fp8)
     else:
         emit({"peaks": {"hbm_gbs": hbm, "fp8_tflops": fp8, "source": src}})
         for m, _, k in inputs.WORKLOAD_SHAPES[2]:
@@ -236,6 +259,8 @@ def main():
             run_gemm_ue8m0(t, dev, m, n, k, a.reps, modes, hbm, fp8)
         for m, n, k in inputs.WORKLOAD_SHAPES[4] + inputs.WORKLOAD_SHAPES[5]:
             run_gemm_pc(t, dev, m, n, k, a.reps, modes, hbm, fp8)
+        for m, n, k in inputs.WORKLOAD_SHAPES[4]:
+            run_linear(t, dev, m, n, k, a.reps, modes, hbm, fp8)
         for m, _, k in inputs.WORKLOAD_SHAPES[3]:
             run_group_ue8m0(t, dev, m, k, a.reps, modes, hbm)
             run_per_channel(t, dev, m, k, a.reps, modes, hbm)

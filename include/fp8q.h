@@ -52,6 +52,7 @@
  *   - Environment: FP8Q_LOG=1 prints the launch chosen for every call to
  *     stderr.  FP8Q_GEMM_TILE forces a GEMM launch mode and
  *     FP8Q_PER_TENSOR_PATH=twopass the two-pass per-tensor path (measurement);
+ *     FP8Q_LINEAR=fused|serial how fp8_linear_group128 runs (measurement);
  *     FP8Q_WAIT_BUDGET_CYCLES bounds the GEMM's device-side waits (fault
  *     testing); both are read once per process.  No environment variable
  *     changes the result of a call that completes.
@@ -145,6 +146,37 @@ int fp8_act_quant_group128(const void* x, int64_t M, int64_t K, int64_t ldx,
  * row-major contiguous; the last row block may hold fewer than 128 rows. */
 int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw,
                               uint8_t* qb, int64_t ldqb, float* sb, void* stream);
+
+/* ------------------------------------------------------------------ */
+/* The dynamic FP8 linear with the activation quantisation fused into   */
+/* the GEMM ([P1] "Analyzing FP8 Quantization Sensitivity": act_quant   */
+/* produces the scales that feed fp8_gemm, and its latency matters at   */
+/* small batch).                                                         */
+/* ------------------------------------------------------------------ */
+
+/* Workspace bytes fp8_linear_group128 needs for (M, N, K) on the current
+ * device (0 when unused; no zero fill needed). */
+size_t fp8_linear_group128_workspace_size(int64_t M, int64_t N, int64_t K);
+
+/* y = block_gemm(act_quant_group128(x), sa; qb, sb): the result of
+ * fp8_act_quant_group128 followed by fp8_block_gemm, bit for bit.
+ *   x : bf16 [M,K] (row stride ldx, a multiple of 8; 16-byte aligned)
+ *   qb: E4M3 [N,K] (row stride ldb), sb: fp32 [ceil(N/128), K/128]
+ *   y : bf16 [M,N] (row stride ldy)
+ * By default the quantisation kernel runs first and the GEMM is launched as
+ * its programmatic dependent: the GEMM starts while the quantisation runs,
+ * issues the weight halves of its first pipeline stages, and waits for the
+ * quantisation only before reading the codes and scales (kept in the
+ * workspace).  With FP8Q_LINEAR=fused, launches that use swapped tiles of
+ * at most 32 tokens quantise each 128-wide K block of the tokens inside the
+ * GEMM instead, writing the codes straight into shared memory (measured
+ * slower on B200: the per-CTA quantisation is repeated by every CTA and
+ * cannot keep pace with the weight stream).  FP8Q_LINEAR=serial runs the two
+ * kernels without overlap.  Every choice gives the same bytes.  Errors as
+ * fp8_block_gemm. */
+int fp8_linear_group128(const void* x, int64_t ldx, const uint8_t* qb, int64_t ldb,
+                        const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                        void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------------------ */
 /* Per-channel scales ([P2] Description names a PER_CHANNEL mode of the */
