@@ -100,6 +100,10 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 8, false, 4>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 7, false, 4>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 1>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true, 1>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<64, true, 8, false, 3>();
@@ -360,7 +364,7 @@ void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR>, tp, tq, tsa, tsb, p);
+    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, tp, tq, tsa, tsb, p);
 }
 
 // ------------------------------------------------------------------ no-alloc GEMM scratch
@@ -676,7 +680,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode != 0);
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2 || mode == 4);   // no ue8m0 / fused pairs
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -727,7 +731,10 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         if (pl.bn == 16) launch_gemm<16, true, 8, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
         else launch_gemm<32, true, 7, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
     } else if (per_channel) {
-        if (pl.swap) {
+        if (pl.pair) {
+            if (pl.bn == 256) launch_gemm<256, false, 6, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+            else launch_gemm<128, false, 8, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else if (pl.swap) {
             switch (pl.bn) {
                 case 16: launch_gemm<16, true, 12, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
                 case 32: launch_gemm<32, true, 10, false, 3>(tp, tq, tsa, tsb, p, pl.grid, st); break;
@@ -757,7 +764,10 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
             launch_gemm<256, false, 4, false, 2>(tp, tq, tsa, tsb, p, pl.grid, st);
         }
     } else if (per_tensor) {
-        if (pl.swap) {
+        if (pl.pair) {
+            if (pl.bn == 256) launch_gemm<256, false, 6, true, 1>(tp, tq, tsa, tsb, p, pl.grid, st);
+            else launch_gemm<128, false, 8, true, 1>(tp, tq, tsa, tsb, p, pl.grid, st);
+        } else if (pl.swap) {
             switch (pl.bn) {
                 case 16: launch_gemm<16, true, 12, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;
                 case 32: launch_gemm<32, true, 10, false, true>(tp, tq, tsa, tsb, p, pl.grid, st); break;

@@ -718,8 +718,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 #pragma unroll
                 for (int ch = 0; ch < kChunks; ++ch) {
                     if constexpr (kChunk == 64) ptx::tmem_ld64(taddr + ch * 64, v);
-                    else if constexpr (kChunk == 32) ptx::tmem_ld32(taddr, v);
-                    else ptx::tmem_ld16(taddr, v);
+                    else if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + ch * 32, v);
+                    else ptx::tmem_ld16(taddr + ch * 16, v);
                     ptx::tmem_wait_ld();
                     if (ch == kChunks - 1) {
                         ptx::tc_fence_before();
