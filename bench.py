@@ -68,27 +68,40 @@ GEMM_SOURCES = ("gemm_kernels.cuh", "ptx_sm100.cuh", "launch_table.inc")
 TRAFFIC_RECORD = os.path.join(ROOT, "profiles", "block_gemm_prefill_4096xNx7168.md")
 
 
+def code_digest(texts) -> str:
+    """sha256 (first 16 hex digits) of C/C++ sources with comments removed
+    and whitespace collapsed: edits to comments or layout keep the digest,
+    any change to the code changes it."""
+    import hashlib
+    import re
+    h = hashlib.sha256()
+    for t in texts:
+        t = re.sub(r"/\*.*?\*/", " ", t, flags=re.S)        # block comments
+        t = re.sub(r"//[^\n]*", " ", t)                      # line comments
+        h.update(" ".join(t.split()).encode())
+    return h.hexdigest()[:16]
+
+
 def gemm_traffic():
     """DRAM bytes per GEMM launch (mean over the step's three launches) from
-    the committed ncu summary -- only while the GEMM sources still hash to the
-    value recorded there; None otherwise."""
-    import hashlib
-    h = hashlib.sha256()
+    the committed ncu summary -- only while the GEMM code still has the
+    digest recorded there; None otherwise."""
     csrc = os.path.join(ROOT, "fp8_dynamic_quantization_b200", "csrc")
     try:
+        texts = []
         for f in GEMM_SOURCES:
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(fh.read())
+            with open(os.path.join(csrc, f)) as fh:
+                texts.append(fh.read())
         rec = {}
         with open(TRAFFIC_RECORD) as fh:
             for line in fh:
                 if ":" in line and line.split(":", 1)[0].strip() in (
-                        "gemm_source_sha256_16", "dram_bytes_per_launch_mean"):
+                        "gemm_code_digest", "dram_bytes_per_launch_mean"):
                     k, v = line.split(":", 1)
                     rec[k.strip()] = v.split()[0]
     except OSError:
         return None
-    if rec.get("gemm_source_sha256_16") != h.hexdigest()[:16]:
+    if rec.get("gemm_code_digest") != code_digest(texts):
         return None
     return float(rec["dram_bytes_per_launch_mean"])
 

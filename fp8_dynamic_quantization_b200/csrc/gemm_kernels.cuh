@@ -16,27 +16,36 @@
 // Warp roles (one CTA per SM, persistent over work units):
 //   warpgroup 0   warp 0: TMA producer (P and Q tiles of one K block per
 //                 pipeline stage); warp 1: TMEM allocation and the single
-//                 thread that issues tcgen05.mma; warps 2-3 idle.  With
-//                 several promotion warpgroups it hands registers to them
+//                 thread that issues tcgen05.mma; warps 2-3: the ue8m0
+//                 scale-slot writer (warp 2, scale mode 2) or the token
+//                 quantisers (scale mode 4), otherwise idle.  With several
+//                 promotion warpgroups warpgroup 0 hands registers to them
 //                 (setmaxnreg 48/224 or 56/216 for two, 32/160 for three).
 //   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row)
-//                 and a slice of kCW <= 64 accumulator columns; warpgroup
-//                 w-1 owns columns [(w-1)*kCW, w*kCW).  Each K block costs a
-//                 thread one tcgen05.ld and one wait before it releases the
-//                 TMEM buffer, which keeps the MMA <-> promotion hand-off
-//                 short; more warpgroups hide the load latency.
+//                 and a slice of kCW accumulator columns (128 for 256-wide
+//                 tiles, else at most 64); warpgroup w-1 owns columns
+//                 [(w-1)*kCW, w*kCW).  A thread loads its slice in chunks
+//                 of at most 64 columns and releases the TMEM buffer as
+//                 soon as the last chunk has landed.
 //
 // Operand roles.  The MMA computes D[128 rows, BN cols] = P * Q^T with P and
 // Q K-major tiles in shared memory (128-byte swizzle).
 //   normal  (SWAP = false): P = A rows (m), Q = B rows (n).  Row scale
 //           sa[m,kb]; column scale sb[n/128,kb] is uniform per 128 columns.
+//           With SS the producer also copies each group of 4 K blocks'
+//           scales (a 128 x 4 fp32 box of sa and the tile's sb rows) into
+//           a shared-memory ring, so the promotion never waits on a global
+//           load.
 //   swapped (SWAP = true) : P = B rows (n), Q = A rows (m), for skinny M --
 //           the weight fills the 128-row MMA dimension and the few tokens
 //           become the MMA's N.  The per-column scale sa[m,kb]*sb[tile,kb]
 //           is computed once per work unit into shared memory.
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
-//
+// Programmatic dependent launch (p.pdl): the producer issues the weight
+// halves of its first STAGES stages, then waits for the grid that writes A
+// and sa (griddepcontrol.wait); the promotion waits before reading scales.
+
 // Scale mode SM:
 //   0  fp32 block scales, promoted per K block as above.
 //   1  per-tensor scales (the GEMM of the per-tensor dynamic path): sa and
@@ -45,7 +54,7 @@
 //   2  ue8m0 block scales (E8M0 bytes sa [M, G], sb [ceil(N/128), G]): the
 //      tensor cores apply them (tcgen05.mma kind::mxf8f6f4.block_scale), so
 //      again one TMEM accumulation per unit and no promotion.  Per group of 4
-//      K blocks the producer warp writes the tile's scale bytes into a
+//      K blocks warp 2 writes the tile's scale bytes into a
 //      shared-memory slot laid out as 32 rows x 16 bytes per 128 rows
 //      (row j holds rows j, 32+j, 64+j, 96+j, four K blocks each); the MMA
 //      warp copies each such block to TMEM with tcgen05.cp 32x128b.warpx4,
@@ -345,63 +354,62 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     // registers per lane (a unit spans <= 64 K blocks) and are fetched by
     // shuffle.
     auto quantise = [&](uint32_t mine) {
-            const int c = lane & 15;
-            const int r0 = lane >> 4;
-
-            uint32_t it = 0, qg = 0;
-            bool stop = false;
-            for (int u = unit0; u < p.units && !stop; u += unit_step) {
-                int tp, tq, kb0, kb1;
-                unit_coords(p, u, tp, tq, kb0, kb1);
-                const float* sbr = p.sb + int64_t(tp) * p.G;
-                const float sb_lo = kb0 + lane < kb1 ? __ldg(sbr + kb0 + lane) : 0.0f;
-                const float sb_hi = kb0 + 32 + lane < kb1 ? __ldg(sbr + kb0 + 32 + lane) : 0.0f;
-                for (int kb = kb0; kb < kb1; ++kb, ++it, ++qg) {
-                    if (it % kQuantWarps != mine) continue;               // another warp's block
-                    const int s = it % STAGES;
-                    const uint32_t ph = (it / STAGES) & 1;
-                    const uint32_t slot = qg % kFqN, sph = (qg / kFqN) & 1;
-                    const int kbl = kb - kb0;
-                    const float sbv = __shfl_sync(0xFFFFFFFFu, kbl < 32 ? sb_lo : sb_hi, kbl & 31);
-                    bool ok = true;
-                    // the tile landing implies the stage's operand slot is free
-                    // (its copy was issued after the stage emptied)
-                    if (lane == 0)
-                        ok = ptx::mbar_wait(&xfull[s], ph, p.wait_budget) &&
-                             ptx::mbar_wait(&qempty[slot], sph ^ 1, p.wait_budget);
-                    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                    if (!ok) { if (lane == 0) fail(); stop = true; break; }
-                    __syncwarp();
-                    const uint8_t* xs = xring + size_t(s) * C::kXBytes;              // BN rows x 256 B
-                    uint8_t* qdst = tiles + size_t(s) * C::kStageBytes + C::kPBytes;   // BN rows x 128 B
-                    // rows r0, r0+2, ...: independent chains, interleaved by full unrolling
-                    constexpr int kRows = BN / 2;
-                    uint4 v[kRows];
-                    uint32_t a[kRows];
+        const int c = lane & 15;
+        const int r0 = lane >> 4;
+        uint32_t it = 0, qg = 0;
+        bool stop = false;
+        for (int u = unit0; u < p.units && !stop; u += unit_step) {
+            int tp, tq, kb0, kb1;
+            unit_coords(p, u, tp, tq, kb0, kb1);
+            const float* sbr = p.sb + int64_t(tp) * p.G;
+            const float sb_lo = kb0 + lane < kb1 ? __ldg(sbr + kb0 + lane) : 0.0f;
+            const float sb_hi = kb0 + 32 + lane < kb1 ? __ldg(sbr + kb0 + 32 + lane) : 0.0f;
+            for (int kb = kb0; kb < kb1; ++kb, ++it, ++qg) {
+                if (it % kQuantWarps != mine) continue;               // another warp's block
+                const int s = it % STAGES;
+                const uint32_t ph = (it / STAGES) & 1;
+                const uint32_t slot = qg % kFqN, sph = (qg / kFqN) & 1;
+                const int kbl = kb - kb0;
+                const float sbv = __shfl_sync(0xFFFFFFFFu, kbl < 32 ? sb_lo : sb_hi, kbl & 31);
+                bool ok = true;
+                // the tile landing implies the stage's operand slot is free
+                // (its copy was issued after the stage emptied)
+                if (lane == 0)
+                    ok = ptx::mbar_wait(&xfull[s], ph, p.wait_budget) &&
+                         ptx::mbar_wait(&qempty[slot], sph ^ 1, p.wait_budget);
+                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+                if (!ok) { if (lane == 0) fail(); stop = true; break; }
+                __syncwarp();
+                const uint8_t* xs = xring + size_t(s) * C::kXBytes;              // BN rows x 256 B
+                uint8_t* qdst = tiles + size_t(s) * C::kStageBytes + C::kPBytes;   // BN rows x 128 B
+                // rows r0, r0+2, ...: independent chains, interleaved by full unrolling
+                constexpr int kRows = BN / 2;
+                uint4 v[kRows];
+                uint32_t a[kRows];
 #pragma unroll
-                    for (int i = 0; i < kRows; ++i) {
-                        v[i] = *reinterpret_cast<const uint4*>(xs + (r0 + 2 * i) * 256 + c * 16);
-                        a[i] = absmax8(v[i]);
-                    }
-#pragma unroll
-                    for (int o = 8; o >= 1; o >>= 1)
-#pragma unroll
-                        for (int i = 0; i < kRows; ++i) a[i] = max(a[i], __shfl_xor_sync(0xFFFFFFFFu, a[i], o));
-#pragma unroll
-                    for (int i = 0; i < kRows; ++i) {
-                        const int r = r0 + 2 * i;
-                        const float sc = scale_from_amax_bits(a[i]);
-                        // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r % 8)
-                        *reinterpret_cast<uint2*>(qdst + r * 128 + ((((c >> 1) ^ (r & 7)) << 4) | ((c & 1) << 3))) =
-                            quant8(v[i], make_scale(sc));
-                        if (c == 0) slab[slot * BN + r] = sc * sbv;
-                    }
-                    ptx::fence_proxy_async_shared();
-                    __syncwarp();
-                    if (lane == 0) { ptx::mbar_arrive(&full[s]); ptx::mbar_arrive(&qfull[slot]); }
+                for (int i = 0; i < kRows; ++i) {
+                    v[i] = *reinterpret_cast<const uint4*>(xs + (r0 + 2 * i) * 256 + c * 16);
+                    a[i] = absmax8(v[i]);
                 }
+#pragma unroll
+                for (int o = 8; o >= 1; o >>= 1)
+#pragma unroll
+                    for (int i = 0; i < kRows; ++i) a[i] = max(a[i], __shfl_xor_sync(0xFFFFFFFFu, a[i], o));
+#pragma unroll
+                for (int i = 0; i < kRows; ++i) {
+                    const int r = r0 + 2 * i;
+                    const float sc = scale_from_amax_bits(a[i]);
+                    // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r % 8)
+                    *reinterpret_cast<uint2*>(qdst + r * 128 + ((((c >> 1) ^ (r & 7)) << 4) | ((c & 1) << 3))) =
+                        quant8(v[i], make_scale(sc));
+                    if (c == 0) slab[slot * BN + r] = sc * sbv;
+                }
+                ptx::fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) { ptx::mbar_arrive(&full[s]); ptx::mbar_arrive(&qfull[slot]); }
             }
-            __syncwarp();
+        }
+        __syncwarp();
     };
 
     if (warp < 4) {
