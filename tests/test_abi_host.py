@@ -116,3 +116,37 @@ def test_python_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(_abi, "_lib", None)
     with pytest.raises(OSError):
         _abi.load()
+
+
+@pytest.mark.parametrize("name", ["fp8_gemm_per_tensor", "fp8_gemm_per_channel", "fp8_block_gemm_ue8m0"])
+def test_scaled_gemm_variants_argument_checks(cuda_lib, name):
+    """The per-tensor, per-channel and ue8m0 GEMMs validate like fp8_block_gemm;
+    only the ue8m0 one accepts byte-aligned scale pointers."""
+    f = getattr(cuda_lib, name)
+    assert f(A, 200, B, C, 200, D, A, 64, 16, 64, 200, None, 0, None) == SHAPE     # K % 128
+    assert f(A, 256, B, C, 256, D, A, 64, 0, 64, 256, None, 0, None) == OK          # empty M
+    assert f(None, 256, B, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == INVALID
+    assert f(A, 256, None, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == INVALID
+    assert f(A, 128, B, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == INVALID    # lda < K
+    assert f(A, 264, B, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == MISALIGNED  # lda pitch
+    odd_scales = f(A, 256, B + 1, C, 256, D + 1, A, 64, 16, 64, 256, None, 0, None)
+    if name == "fp8_block_gemm_ue8m0":
+        assert odd_scales != MISALIGNED
+    else:
+        assert odd_scales == MISALIGNED
+
+
+def test_linear_group128_argument_checks(cuda_lib):
+    f = cuda_lib.fp8_linear_group128
+    assert f(A, 200, C, 200, D, B, 64, 16, 64, 200, None, 0, None) == SHAPE        # K % 128
+    assert f(A, 256, C, 256, D, B, 64, 0, 64, 256, None, 0, None) == OK            # empty M
+    assert f(A, 256, C, 256, D, B, 64, -1, 64, 256, None, 0, None) == INVALID
+
+
+@pytest.mark.parametrize("name", ["fp8_act_quant_per_channel", "fp8_act_quant_group128_ue8m0"])
+def test_new_quant_argument_checks(cuda_lib, name):
+    f = getattr(cuda_lib, name)
+    assert f(A, 4, 130, 130, B, 136, C, None) == SHAPE                             # K % 8 / % 128
+    assert f(A, 4, 256, 256, B, 256, None, None) == INVALID
+    assert f(A + 8, 4, 256, 256, B, 256, C, None) == MISALIGNED
+    assert f(A, 0, 256, 256, B, 256, C, None) == OK                                # empty
