@@ -296,11 +296,12 @@ int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa,
 /* ------------------------------------------------------------------ */
 
 /* The pages have no counterpart to this call; it exists for callers that
- * cannot allocate device memory: code running while a stream is being
- * captured (where cudaMalloc is not allowed), host frameworks and plugin
- * interfaces that hand a kernel only its input and output buffers, and
- * latency-critical loops that cannot afford cudaMalloc/cudaFree (cudaFree
- * synchronises the device).
+ * cannot allocate device memory: host frameworks and plugin interfaces that
+ * hand a kernel only its input and output buffers and own every other byte
+ * of the device; serving processes that reserve the whole device pool at
+ * start-up, so that a later cudaMalloc would fail; and latency-critical
+ * loops that cannot afford cudaMalloc/cudaFree (cudaFree synchronises the
+ * device).
  *
  * Same operation, arguments, layouts and errors as fp8_block_gemm, minus
  * the workspace.  The split-K partial sums that fp8_block_gemm would put in

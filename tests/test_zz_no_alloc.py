@@ -1,6 +1,7 @@
 """fp8_block_gemm_noalloc: the block GEMM for callers that cannot allocate
-device memory (code running under stream capture, plugin hosts that hand over
-only input and output buffers, loops that cannot pay for cudaMalloc/cudaFree).
+device memory (plugin hosts that hand over only input and output buffers,
+serving processes that reserve the whole device pool at start-up, loops that
+cannot pay for cudaMalloc/cudaFree).
 Its split-K scratch is a fixed array inside the library instead of a caller
 workspace.
 
