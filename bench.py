@@ -409,7 +409,8 @@ def our_arm(args, rank, world, local_rank):
                          "traffic": gemm_traffic(),
                          "traffic_unit": "bytes per GEMM launch (mean of the step's 3), ncu",
                          "algorithmic_bytes_per_launch": sum(bytes_gemm(M, n) for n in NS) / len(NS),
-                         "kernel": "block_gemm_kernel (all three N per step)",
+                         "kernel": "block_gemm_kernel (all three N per step; at N=7168 the call's "
+                                   "time includes tail_reduce_kernel, which sums the split last wave)",
                          "peak_source": f"{peak_src} bf16 "
                                         f"{'burst' if timed_s < 5.0 else 'sustained'} x {FP8_OVER_BF16} (fp8/bf16 nominal)"},
             "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

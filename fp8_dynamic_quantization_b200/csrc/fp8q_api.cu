@@ -168,6 +168,7 @@ const TableRow kGemmTable[] = {
 struct GemmPlan {
     bool swap, pair;
     int bn, stages, splits, tiles_p, tiles_q, units, grid;
+    int full_tiles, tail_tiles, tail_splits;   // split tail (normal tiles only)
     int64_t ldw;
     size_t ws_bytes;
 };
@@ -225,7 +226,17 @@ bool tile_override(TableRow* out) {
 
 // Only the fp32 block-scaled GEMM has a CTA-pair variant: for the others a
 // forced pair row runs as the single-CTA tile of the same width.
-GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = false) {
+//
+// Split tail: with one whole tile per unit, a tile count just above a
+// multiple of the SM count leaves a last wave in which few SMs work for a
+// whole tile time (4096 x 7168 with 128 x 256 tiles: 896 tiles = 6 waves of
+// 148 + 8).  If that last wave holds at most half the SMs, its tiles are
+// split along K into S = min(SMs / tail, K blocks / 2) ranges instead, so it
+// takes about 1/S of a tile time; tail_reduce_kernel then adds the S fp32
+// partials of each tail tile in fixed order.  ws_cap bounds the workspace
+// this may use (S shrinks to fit; below 2 the tail stays whole).
+GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = false,
+                   size_t ws_cap = ~size_t(0)) {
     GemmPlan pl{};
     const TableRow* row = &kGemmTable[0];
     for (const TableRow& r : kGemmTable)
@@ -256,10 +267,26 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
     }
     pl.splits = splits;
     pl.units = int(tiles * splits);
+    pl.full_tiles = int(tiles);
+    pl.tail_tiles = 0;
+    pl.tail_splits = 1;
+    if (!pl.swap && !pl.pair && splits == 1 && tiles > sms && tiles % sms != 0) {
+        const int tail = int(tiles % sms);
+        const size_t slot_bytes = size_t(tail) * 128 * size_t(pl.bn) * sizeof(float);   // one split of every tail tile
+        const int s = int(std::min<size_t>(size_t(std::min(sms / tail, G / 2)), ws_cap / slot_bytes));
+        if (s >= 2) {
+            pl.tail_tiles = tail;
+            pl.tail_splits = s;
+            pl.full_tiles = int(tiles) - tail;
+            pl.units = pl.full_tiles + tail * s;
+        }
+    }
     pl.grid = pl.pair ? 2 * std::max(1, std::min(pl.units, sms / 2))
                       : std::max(1, std::min(pl.units, sms));
     pl.ldw = (N + 7) / 8 * 8;
-    pl.ws_bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(pl.ldw) * sizeof(float) : 0;
+    pl.ws_bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(pl.ldw) * sizeof(float)
+                : pl.tail_tiles > 0 ? size_t(pl.tail_tiles) * size_t(pl.tail_splits) * 128 * size_t(pl.bn) * sizeof(float)
+                : 0;
     return pl;
 }
 
@@ -647,7 +674,8 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != FP8Q_OK) return 0;
-    return plan_gemm(M, N, K, d->sms).ws_bytes;
+    // the ue8m0 and fused GEMMs never run as CTA pairs: size for both plans
+    return std::max(plan_gemm(M, N, K, d->sms).ws_bytes, plan_gemm(M, N, K, d->sms, true).ws_bytes);
 }
 
 }  // extern "C"
@@ -655,7 +683,8 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                     void* workspace, size_t workspace_bytes, void* stream, int mode,
-                    const uint16_t* x = nullptr, int64_t ldx = 0, bool pdl = false) {
+                    const uint16_t* x = nullptr, int64_t ldx = 0, bool pdl = false,
+                    size_t ws_cap = ~size_t(0)) {
     // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes;
     // 3: per-channel fp32 scales; 4: fp32 block scales with the group-128
     // quantisation of bf16 tokens x fused in (swapped tiles of <= 64 tokens;
@@ -680,7 +709,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2 || mode == 4);   // no ue8m0 / fused pairs
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2 || mode == 4, ws_cap);   // no ue8m0 / fused pairs
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -705,13 +734,13 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     p.N = int(N);
     p.G = int(K / 128);
     p.tiles_p = pl.tiles_p;
-    p.tiles_q = pl.tiles_q;
     p.splits = pl.splits;
     p.units = pl.units;
+    p.full_units = pl.tail_tiles > 0 ? pl.full_tiles : pl.units;
+    p.full_tiles = pl.full_tiles;
+    p.tail_splits = pl.tail_splits;
     p.scale_vec4 = mode == 0 && (p.G % 4 == 0) && aligned16(sa) && aligned16(sb);
     p.sf_words = ue8m0 && (p.G % 4 == 0) && aligned4(sa) && aligned4(sb);
-    p.x = x;
-    p.ldx = ldx;
     p.pdl = (pdl && mode == 0 && !pl.pair) ? 1 : 0;
     // Normal 128/256-wide tiles stage the block scales through shared memory
     // (TMA boxes of 4 K blocks) when the scale rows allow 16-byte boxes.
@@ -723,10 +752,11 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     if (fused && !make_x_tmap(&tsa, x, M, K, ldx, pl.bn)) return FP8Q_ERR_CUDA;   // the token tiles
     p.wait_budget = wait_budget_cycles();
     if (log_enabled())
-        std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d\n",
+        std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d"
+                             " tail=%dx%d\n",
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
-                     pl.stages, pl.splits, pl.units, pl.grid);
+                     pl.stages, pl.splits, pl.units, pl.grid, pl.tail_tiles, pl.tail_splits);
     if (fused) {
         if (pl.bn == 16) launch_gemm<16, true, 8, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
         else launch_gemm<32, true, 7, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
@@ -803,6 +833,12 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         const int64_t total = M * ((N + 3) / 4);
         const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
         splitk_reduce_kernel<<<g, 256, 0, st>>>(p.ws, pl.splits, p.M, p.N, pl.ldw, p.y, ldy);
+        rc = launch_status();
+    } else if (pl.tail_tiles > 0) {
+        const int64_t total = int64_t(pl.tail_tiles) * 128 * (pl.bn / 4);
+        const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
+        tail_reduce_kernel<<<g, 256, 0, st>>>(p.ws, pl.tail_tiles, pl.tail_splits, pl.full_tiles,
+                                              pl.tiles_p, pl.bn, p.M, p.N, p.y, ldy);
         rc = launch_status();
     }
     return rc;
@@ -898,12 +934,17 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, cons
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 || N == 0) return FP8Q_OK;
-    if (fp8_block_gemm_workspace_size(M, N, K) > kNoAllocScratchBytes) return FP8Q_ERR_WORKSPACE;
-    void* scratch = nullptr;
-    const int rc = noalloc_scratch(&scratch);
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
-    return fp8_block_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, scratch, kNoAllocScratchBytes,
-                          stream);
+    // regular split-K partials must fit the scratch; a split tail is cut to fit it
+    if (plan_gemm(M, N, K, d->sms, false, kNoAllocScratchBytes).ws_bytes > kNoAllocScratchBytes)
+        return FP8Q_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    rc = noalloc_scratch(&scratch);
+    if (rc != FP8Q_OK) return rc;
+    return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, scratch, kNoAllocScratchBytes, stream, 0,
+                    nullptr, 0, false, kNoAllocScratchBytes);
 }
 
 // ------------------------------------------------------------ status

@@ -42,6 +42,12 @@
 //           is computed once per work unit into shared memory.
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
+// Split tail (normal tiles): when the tiles leave a last wave that would
+// occupy only a few SMs, the first full_tiles tiles run whole and each of
+// the remaining tail tiles is split into tail_splits K ranges, so the last
+// wave is short and fills the SMs; those partials go to the workspace
+// (tile-local [unit][128][BN] fp32) and tail_reduce_kernel adds them in
+// fixed order into Y.
 // Programmatic dependent launch (p.pdl): the producer issues the weight
 // halves of its first STAGES stages, then waits for the grid that writes A
 // and sa (griddepcontrol.wait); the promotion waits before reading scales.
@@ -66,7 +72,8 @@
 //      TMEM accumulation per unit; the epilogue multiplies row m by its
 //      scale and column n by the one staged for the tile in shared memory.
 //   4  swapped mode with the group-128 quantisation of the tokens fused in:
-//      A arrives as bf16 (p.x).  The producer also copies each K block's bf16
+//      A arrives as bf16 (read through the token tensor map, the tmSA
+//      argument).  The producer also copies each K block's bf16
 //      token tile (BN rows x 256 bytes) into a per-stage ring; warps 2-3
 //      quantise it (per-row amax over the block = the 1x128 group, scale =
 //      amax/448, codes), write the codes into the stage's operand slot in
@@ -85,17 +92,22 @@ struct GemmParams {
     const float* sa;     // [M, G]
     const float* sb;     // [ceil(N/128), G]
     uint16_t* y;         // bf16 [M, ldy]
-    float* ws;           // split-K partials [splits, M, ldw]
+    float* ws;           // split-K partials [splits, M, ldw], or the split tail's
     int64_t ldy, ldw;
     int M, N, G;
-    int tiles_p, tiles_q, splits, units;
-    int scale_vec4;      // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
-    int sf_words;        // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
-    const uint16_t* x;   // fused quantisation: bf16 tokens [M, ldx]
-    int64_t ldx;
-    int pdl;             // launched as a programmatic dependent of the kernel producing A and sa
+    int tiles_p, splits, units;
+    int full_units;      // units [0, full_units): tiles x splits; the rest are split-tail units
+    int full_tiles;      // tiles before the split tail
+    int tail_splits;     // K ranges per tail tile; their partials go to ws as [unit - full_units][128][BN]
+    // Flags as bytes and no field the kernel does not read: the struct is
+    // passed by value to every launch, and growing it from 120 to 136
+    // bytes measurably slowed the kernel (2%).
+    uint8_t scale_vec4;  // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
+    uint8_t sf_words;    // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
+    uint8_t pdl;         // launched as a programmatic dependent of the kernel producing A and sa
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
+static_assert(sizeof(GemmParams) <= 104, "GemmParams size");
 
 template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 struct GemmCfg {
@@ -164,12 +176,21 @@ struct GemmCfg {
 
 __device__ __forceinline__ void unit_coords(const GemmParams& p, int u, int& tp, int& tq,
                                             int& kb0, int& kb1) {
-    const int split = u % p.splits;
-    const int tile = u / p.splits;
+    int split, tile, splits;
+    if (u < p.full_units) {
+        splits = p.splits;
+        split = u % splits;
+        tile = u / splits;
+    } else {                                   // split tail
+        splits = p.tail_splits;
+        const int v = u - p.full_units;
+        split = v % splits;
+        tile = p.full_tiles + v / splits;
+    }
     tp = tile % p.tiles_p;
     tq = tile / p.tiles_p;
-    kb0 = int((int64_t(split) * p.G) / p.splits);
-    kb1 = int((int64_t(split + 1) * p.G) / p.splits);
+    kb0 = int((int64_t(split) * p.G) / splits);
+    kb1 = int((int64_t(split + 1) * p.G) / splits);
 }
 
 // Accumulators are kept as packed fp32 pairs: acc2[i] holds columns 2i and
@@ -756,7 +777,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 #pragma unroll
                 for (int j = 0; j < C::kCW; ++j) acc[j] *= slab[chalf * C::kCW + j];
             }
-            if (p.splits == 1) {
+            if (p.splits == 1 && u < p.full_units) {
                 if (!SWAP) {
                     const int m = m_row;
                     const int n_first = q0 + chalf * C::kCW;
@@ -793,13 +814,18 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     }
                 }
             } else {
+                // fp32 partial: split-K slot [split][M][ldw], or (split tail,
+                // normal tiles) slot u - full_units laid out [128][BN] per tile
+                const bool tail = u >= p.full_units;
                 const int split = u % p.splits;
                 float* wsp = p.ws + int64_t(split) * p.M * p.ldw;
                 if (!SWAP) {
                     const int m = m_row;
                     const int n_first = q0 + chalf * C::kCW;
                     if (m < p.M) {
-                        float* wr = wsp + int64_t(m) * p.ldw;
+                        // row m, indexed by the output column n
+                        float* wr = tail ? p.ws + (int64_t(u - p.full_units) * 128 + row) * BN - q0
+                                         : wsp + int64_t(m) * p.ldw;
 #pragma unroll
                         for (int j = 0; j < C::kCW; j += 4) {
                             const int n = n_first + j;
@@ -864,6 +890,42 @@ splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int
             for (int s = 0; s < splits; ++s)
                 for (int t = 0; t < 4 && n + t < N; ++t)
                     a[t] += ws[(int64_t(s) * M + m) * ldw + n + t];
+            for (int t = 0; t < 4 && n + t < N; ++t)
+                y[m * ldy + n + t] = uint16_t(ptx::pack_bf16x2(a[t], 0.0f) & 0xFFFF);
+        }
+    }
+}
+
+// Fixed-order sum of the split-tail partials (slot tt * splits + s holds
+// split s of tail tile tt, 128 x bn fp32) and conversion to bf16 into Y.
+// Each thread handles 4 consecutive columns of one tile row.
+__global__ void __launch_bounds__(256)
+tail_reduce_kernel(const float* __restrict__ ws, int tail_tiles, int splits, int full_tiles, int tiles_p,
+                   int bn, int M, int N, uint16_t* __restrict__ y, int64_t ldy) {
+    const int quads = bn / 4;
+    const int64_t per_tile = int64_t(128) * quads;
+    const int64_t total = int64_t(tail_tiles) * per_tile;
+    for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < total; i += int64_t(gridDim.x) * 256) {
+        const int tt = int(i / per_tile);
+        const int rem = int(i - int64_t(tt) * per_tile);
+        const int r = rem / quads;
+        const int c = (rem - r * quads) * 4;
+        const int tile = full_tiles + tt;
+        const int64_t m = int64_t(tile % tiles_p) * 128 + r;
+        const int n = (tile / tiles_p) * bn + c;
+        if (m >= M || n >= N) continue;
+        const float* src = ws + (int64_t(tt) * splits * 128 + r) * bn + c;
+        float a[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int s = 0; s < splits; ++s) {
+            const float4 v = __ldcs(reinterpret_cast<const float4*>(src + int64_t(s) * 128 * bn));
+            a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+        }
+        if (n + 4 <= N) {
+            uint2 o;
+            o.x = ptx::pack_bf16x2(a[0], a[1]);
+            o.y = ptx::pack_bf16x2(a[2], a[3]);
+            *reinterpret_cast<uint2*>(y + m * ldy + n) = o;
+        } else {
             for (int t = 0; t < 4 && n + t < N; ++t)
                 y[m * ldy + n + t] = uint16_t(ptx::pack_bf16x2(a[t], 0.0f) & 0xFFFF);
         }

@@ -230,8 +230,8 @@ int fp8_weight_quant_block128_ue8m0(const void* w, int64_t N, int64_t K, int64_t
 /* ------------------------------------------------------------------ */
 
 /* Bytes of device workspace fp8_block_gemm needs for (M, N, K) on the
- * current device (split-K partial sums for skinny M; 0 when unused).
- * The workspace needs no zero fill. */
+ * current device (split-K partial sums for skinny M, or those of a split
+ * last wave; 0 when unused).  The workspace needs no zero fill. */
 size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* Y = A * B^T with block scales:
@@ -244,7 +244,11 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  *   y : bf16 [M,N], row stride ldy
  * K must be a multiple of 128; M, N >= 0 arbitrary (tails handled).
  * The launch (tile shape, operand swap, split-K) is chosen per shape from
- * a compiled table.  Bounded device waits report FP8Q_ERR_TIMEOUT through
+ * a compiled table.  When whole 128-row tiles would leave a last wave that
+ * fills at most half the SMs, the tiles of that wave are split along K and
+ * their fp32 partials are added in fixed order by a second kernel (the
+ * call then enqueues two kernels); results are deterministic for a given
+ * shape and device.  Bounded device waits report FP8Q_ERR_TIMEOUT through
  * fp8q_device_status. */
 int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                    const uint8_t* qb, int64_t ldb, const float* sb,
@@ -311,7 +315,10 @@ int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa,
  * whose launch needs more scratch than that (fp8_block_gemm_workspace_size
  * (M,N,K) > FP8Q_NOALLOC_MAX_SCRATCH_BYTES) are rejected with
  * FP8Q_ERR_WORKSPACE before anything is enqueued; use fp8_block_gemm for
- * them.
+ * them.  The one exception is a split last wave (see fp8_block_gemm): its
+ * tiles are split into fewer K ranges when the scratch is too small for the
+ * split fp8_block_gemm would use, so the bytes of those tiles can differ
+ * from fp8_block_gemm's in rounding, within the same tolerance.
  *
  * The call allocates nothing: no cudaMalloc, cudaFree or allocating
  * library routine.  The first call on each device looks up the scratch

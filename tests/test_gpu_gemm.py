@@ -106,6 +106,58 @@ def test_gemm_prefill_shapes(oracle_mod, gpu, n):
     assert_within(oracle_mod, y_f64(y)[ms, ns], R, T, f"prefill 4096x{n}")
 
 
+def tail_region(M, N, K, sms):
+    """Rows and columns of the tiles the planner splits along K (128 x 256
+    tiles past the last full wave of `sms` CTAs, when that last wave fills at
+    most half the SMs); empty when no tile is split."""
+    tiles_p, tiles_q = -(-M // 128), -(-N // 256)
+    tiles = tiles_p * tiles_q
+    tail = tiles % sms
+    if M <= 512 or tiles <= sms or tail == 0 or min(sms // tail, (K // 128) // 2) < 2:
+        return []
+    out = []
+    for t in range(tiles - tail, tiles):
+        tp, tq = t % tiles_p, t // tiles_p
+        out.append((np.arange(tp * 128, min(M, tp * 128 + 128)), np.arange(tq * 256, min(N, tq * 256 + 256))))
+    return out
+
+
+def region_points(region):
+    ms, ns = [], []
+    for rows, cols in region:
+        mm, nn = np.meshgrid(rows, cols, indexing="ij")
+        ms.append(mm.ravel())
+        ns.append(nn.ravel())
+    return np.concatenate(ms), np.concatenate(ns)
+
+
+@pytest.mark.parametrize("m,n,k", [(4096, 7168, 7168), (4000, 7100, 1024)])
+def test_gemm_split_tail_tiles(oracle_mod, gpu, m, n, k):
+    """Shapes whose tiles leave a short last wave: those tiles run split
+    along K and are summed by the tail reduce (launch count 2).  Every output
+    of the split tiles (ragged rows and columns in the second shape) and
+    sampled points elsewhere against the oracle; two calls give the same
+    bytes."""
+    sms = torch.cuda.get_device_properties(gpu).multi_processor_count
+    region = tail_region(m, n, k, sms)
+    assert region, "shape chosen to split its last wave"
+    qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m + n + k)
+    before = fq.library().fp8q_launch_count()
+    y = run_gemm(qa, sa, qb, sb, gpu)
+    torch.cuda.synchronize()
+    assert fq.library().fp8q_launch_count() - before == 2
+    Y = y_f64(y)
+    ms, ns = region_points(region)
+    R, T = oracle_mod.block_gemm_points(qa, sa, qb, sb, ms, ns)
+    assert_within(oracle_mod, Y[ms, ns], R, T, f"split tail {m}x{n}x{k}")
+    ms, ns = sample_points(m, n, np.random.default_rng(k))
+    R, T = oracle_mod.block_gemm_points(qa, sa, qb, sb, ms, ns)
+    assert_within(oracle_mod, Y[ms, ns], R, T, f"{m}x{n}x{k}")
+    y2 = run_gemm(qa, sa, qb, sb, gpu)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))     # deterministic
+    assert fq.device_status() == 0
+
+
 def test_gemm_tiny_linear_layer_end_to_end(oracle_mod, gpu):
     """bf16 X[64,2048] and W[2048,2048]: GPU quantisation of both, then the
     GEMM, against the oracle's quantisation (bit-exact) and GEMM."""

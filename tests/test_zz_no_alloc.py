@@ -56,6 +56,40 @@ def test_noalloc_matches_allocating_gemm_twice(oracle_mod, cuda_lib, gpu, m, n, 
     assert fq.device_status() == 0
 
 
+def test_noalloc_cuts_the_split_tail_to_its_scratch(oracle_mod, cuda_lib, gpu):
+    """4000 x 7100 x 4608 leaves a short last wave whose tiles the GEMM splits
+    along K; the allocating call's split needs more than the fixed scratch,
+    so this call splits them fewer ways.  Tiles outside that wave are
+    computed the same way by both calls (same bytes); the split tiles are
+    checked against the oracle's tolerance.  Two calls in a row."""
+    lib = _abi.load()
+    m, n, k = 4000, 7100, 4608
+    assert lib.fp8_block_gemm_workspace_size(m, n, k) > _abi.NOALLOC_MAX_SCRATCH_BYTES
+    sms = torch.cuda.get_device_properties(gpu).multi_processor_count
+    tiles_p, tiles_q = -(-m // 128), -(-n // 256)
+    tail = (tiles_p * tiles_q) % sms
+    assert 0 < tail <= sms // 2
+    in_tail = np.zeros((m, n), dtype=bool)
+    for t in range(tiles_p * tiles_q - tail, tiles_p * tiles_q):
+        tp, tq = t % tiles_p, t // tiles_p
+        in_tail[tp * 128:tp * 128 + 128, tq * 256:tq * 256 + 256] = True
+    ms, ns = np.nonzero(in_tail)
+    for seed in (303, 404):
+        qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=seed)
+        tqa, tsa, tqb, tsb = (_dev(a, gpu) for a in (qa, sa, qb, sb))
+        ldy = (n + 7) // 8 * 8                 # 16-byte row pitch
+        y = torch.full((m, ldy), float("nan"), dtype=torch.bfloat16, device=gpu)[:, :n]
+        assert _noalloc(lib, tqa, tsa, tqb, tsb, y) == FP8Q_OK
+        y_ref = fq.block_gemm(tqa, tsa, tqb, tsb)
+        torch.cuda.synchronize()
+        Y = y.float().cpu().numpy().astype(np.float64)
+        Yr = y_ref.float().cpu().numpy().astype(np.float64)
+        assert np.array_equal(Y[~in_tail], Yr[~in_tail])
+        R, T = oracle_mod.block_gemm_points(qa, sa, qb, sb, ms, ns)
+        assert np.all(np.abs(Y[ms, ns] - R) <= oracle_mod.gemm_tolerance(R, T)), f"seed {seed}"
+    assert fq.device_status() == 0
+
+
 def test_noalloc_rejects_shapes_beyond_its_scratch(cuda_lib, gpu):
     lib = _abi.load()
     m, n, k = 120, 2048, 7168
