@@ -777,7 +777,61 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 #pragma unroll
                 for (int j = 0; j < C::kCW; ++j) acc[j] *= slab[chalf * C::kCW + j];
             }
-            if (p.splits == 1 && u < p.full_units) {
+            if (p.splits == 1 && u < p.full_units && !SWAP && C::kCW % 64 == 0) {
+                // Coalesced bf16 stores.  Within each group of 8 lanes (8 tile
+                // rows), an 8 x 8 transpose of 16-byte chunks per 64-column
+                // block (three butterfly stages of shuffles) leaves lane g of
+                // the group with chunk g of each of the 8 rows, so store k
+                // writes row (group base + k) as 128 contiguous bytes: a warp
+                // store covers 4 whole rows' lines instead of 32 rows' 16-byte
+                // pieces.  Writing a tile row by row took ~8000 clocks per tile
+                // with the MMA stalled behind it; this takes ~3200.
+                const int g8 = lane & 7;
+                const int m_base = tp * C::kTileRows + int(rank) * 128 + quarter * 32 + (lane & ~7);
+#pragma unroll
+                for (int b = 0; b < C::kCW / 64; ++b) {
+                    uint4 a[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int j = b * 64 + k * 8;
+                        a[k].x = ptx::pack_bf16x2(acc[j + 0], acc[j + 1]);
+                        a[k].y = ptx::pack_bf16x2(acc[j + 2], acc[j + 3]);
+                        a[k].z = ptx::pack_bf16x2(acc[j + 4], acc[j + 5]);
+                        a[k].w = ptx::pack_bf16x2(acc[j + 6], acc[j + 7]);
+                    }
+#pragma unroll
+                    for (int sft = 4; sft >= 1; sft >>= 1) {
+                        const bool up = (g8 & sft) != 0;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (k & sft) continue;
+                            const uint4 snd = up ? a[k] : a[k | sft];
+                            uint4 rcv;
+                            rcv.x = __shfl_xor_sync(0xFFFFFFFFu, snd.x, sft);
+                            rcv.y = __shfl_xor_sync(0xFFFFFFFFu, snd.y, sft);
+                            rcv.z = __shfl_xor_sync(0xFFFFFFFFu, snd.z, sft);
+                            rcv.w = __shfl_xor_sync(0xFFFFFFFFu, snd.w, sft);
+                            if (up) a[k] = rcv;
+                            else a[k | sft] = rcv;
+                        }
+                    }
+                    const int n = q0 + chalf * C::kCW + b * 64 + g8 * 8;     // a[k] = chunk g8 of row m_base + k
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int m = m_base + k;
+                        if (m >= p.M) continue;
+                        uint16_t* yr = p.y + int64_t(m) * p.ldy;
+                        if (n + 8 <= p.N) {
+                            *reinterpret_cast<uint4*>(yr + n) = a[k];
+                        } else {
+                            const uint32_t wv[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+#pragma unroll
+                            for (int t = 0; t < 8; ++t)
+                                if (n + t < p.N) yr[n + t] = uint16_t(wv[t >> 1] >> (16 * (t & 1)));
+                        }
+                    }
+                }
+            } else if (p.splits == 1 && u < p.full_units) {
                 if (!SWAP) {
                     const int m = m_row;
                     const int n_first = q0 + chalf * C::kCW;
