@@ -229,6 +229,32 @@ __device__ __forceinline__ float pick4(const float4& v, int i) {
     return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
 
+// Epilogue stores.  A promotion thread holds one tile row, so storing rows
+// directly makes each warp store touch 32 rows in 16-byte pieces.  Within
+// each group of 8 lanes (8 rows), an 8 x 8 transpose of 16-byte chunks
+// (three butterfly stages of shuffles) turns a[k] = chunk k of this lane's
+// row into a[k] = chunk g8 of row (group base + k); store k then writes
+// that row's 8 chunks (128 contiguous bytes) from the 8 lanes, and a warp
+// store covers 4 whole row segments.  All 32 lanes must call it.
+__device__ __forceinline__ void transpose8x8(uint4 (&a)[8], int g8) {
+#pragma unroll
+    for (int sft = 4; sft >= 1; sft >>= 1) {
+        const bool up = (g8 & sft) != 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            if (k & sft) continue;
+            const uint4 snd = up ? a[k] : a[k | sft];
+            uint4 rcv;
+            rcv.x = __shfl_xor_sync(0xFFFFFFFFu, snd.x, sft);
+            rcv.y = __shfl_xor_sync(0xFFFFFFFFu, snd.y, sft);
+            rcv.z = __shfl_xor_sync(0xFFFFFFFFu, snd.z, sft);
+            rcv.w = __shfl_xor_sync(0xFFFFFFFFu, snd.w, sft);
+            if (up) a[k] = rcv;
+            else a[k | sft] = rcv;
+        }
+    }
+}
+
 // ue8m0 mode: E8M0 bytes of K blocks [4g, 4g+4) for one 128-row block of
 // the P operand (is_p) or the Q operand, packed 4 per word (K block 4g+b in
 // byte b); rows, blocks and K blocks out of range give 127 (scale 1).
@@ -778,14 +804,9 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 for (int j = 0; j < C::kCW; ++j) acc[j] *= slab[chalf * C::kCW + j];
             }
             if (p.splits == 1 && u < p.full_units && !SWAP && C::kCW % 64 == 0) {
-                // Coalesced bf16 stores.  Within each group of 8 lanes (8 tile
-                // rows), an 8 x 8 transpose of 16-byte chunks per 64-column
-                // block (three butterfly stages of shuffles) leaves lane g of
-                // the group with chunk g of each of the 8 rows, so store k
-                // writes row (group base + k) as 128 contiguous bytes: a warp
-                // store covers 4 whole rows' lines instead of 32 rows' 16-byte
-                // pieces.  Writing a tile row by row took ~8000 clocks per tile
-                // with the MMA stalled behind it; this takes ~3200.
+                // bf16 Y, 64 columns (8 chunks) per block, stored through
+                // transpose8x8.  Writing a tile row by row took ~8000 clocks
+                // per tile with the MMA stalled behind it; this takes ~3200.
                 const int g8 = lane & 7;
                 const int m_base = tp * C::kTileRows + int(rank) * 128 + quarter * 32 + (lane & ~7);
 #pragma unroll
@@ -799,22 +820,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                         a[k].z = ptx::pack_bf16x2(acc[j + 4], acc[j + 5]);
                         a[k].w = ptx::pack_bf16x2(acc[j + 6], acc[j + 7]);
                     }
-#pragma unroll
-                    for (int sft = 4; sft >= 1; sft >>= 1) {
-                        const bool up = (g8 & sft) != 0;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            if (k & sft) continue;
-                            const uint4 snd = up ? a[k] : a[k | sft];
-                            uint4 rcv;
-                            rcv.x = __shfl_xor_sync(0xFFFFFFFFu, snd.x, sft);
-                            rcv.y = __shfl_xor_sync(0xFFFFFFFFu, snd.y, sft);
-                            rcv.z = __shfl_xor_sync(0xFFFFFFFFu, snd.z, sft);
-                            rcv.w = __shfl_xor_sync(0xFFFFFFFFu, snd.w, sft);
-                            if (up) a[k] = rcv;
-                            else a[k | sft] = rcv;
-                        }
-                    }
+                    transpose8x8(a, g8);
                     const int n = q0 + chalf * C::kCW + b * 64 + g8 * 8;     // a[k] = chunk g8 of row m_base + k
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -873,11 +879,43 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 const bool tail = u >= p.full_units;
                 const int split = u % p.splits;
                 float* wsp = p.ws + int64_t(split) * p.M * p.ldw;
-                if (!SWAP) {
+                if (!SWAP && C::kCW % 32 == 0) {
+                    // 32 fp32 columns (8 chunks) per block, through transpose8x8
+                    const int g8 = lane & 7;
+                    const int r_base = quarter * 32 + (lane & ~7);          // tile row of a[0] after the transpose
+                    const int m_base = tp * C::kTileRows + int(rank) * 128 + r_base;
+#pragma unroll
+                    for (int b = 0; b < C::kCW / 32; ++b) {
+                        uint4 a[8];
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int j = b * 32 + k * 4;
+                            a[k] = make_uint4(__float_as_uint(acc[j]), __float_as_uint(acc[j + 1]),
+                                              __float_as_uint(acc[j + 2]), __float_as_uint(acc[j + 3]));
+                        }
+                        transpose8x8(a, g8);
+                        const int n = q0 + chalf * C::kCW + b * 32 + g8 * 4;  // a[k] = chunk g8 of row m_base + k
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const int m = m_base + k;
+                            if (m >= p.M) continue;
+                            // row m, indexed by the output column n
+                            float* wr = tail ? p.ws + (int64_t(u - p.full_units) * 128 + r_base + k) * BN - q0
+                                             : wsp + int64_t(m) * p.ldw;
+                            if (n + 4 <= p.N) {
+                                *reinterpret_cast<uint4*>(wr + n) = a[k];
+                            } else {
+                                const uint32_t wv[4] = {a[k].x, a[k].y, a[k].z, a[k].w};
+#pragma unroll
+                                for (int t = 0; t < 4; ++t)
+                                    if (n + t < p.N) wr[n + t] = __uint_as_float(wv[t]);
+                            }
+                        }
+                    }
+                } else if (!SWAP) {
                     const int m = m_row;
                     const int n_first = q0 + chalf * C::kCW;
                     if (m < p.M) {
-                        // row m, indexed by the output column n
                         float* wr = tail ? p.ws + (int64_t(u - p.full_units) * 128 + row) * BN - q0
                                          : wsp + int64_t(m) * p.ldw;
 #pragma unroll
@@ -970,9 +1008,16 @@ tail_reduce_kernel(const float* __restrict__ ws, int tail_tiles, int splits, int
         if (m >= M || n >= N) continue;
         const float* src = ws + (int64_t(tt) * splits * 128 + r) * bn + c;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int s = 0; s < splits; ++s) {
-            const float4 v = __ldcs(reinterpret_cast<const float4*>(src + int64_t(s) * 128 * bn));
-            a[0] += v.x; a[1] += v.y; a[2] += v.z; a[3] += v.w;
+        // loads issued 6 at a time, added in split order
+        for (int s0 = 0; s0 < splits; s0 += 6) {
+            float4 v[6];
+#pragma unroll
+            for (int t = 0; t < 6; ++t)
+                v[t] = s0 + t < splits ? __ldcs(reinterpret_cast<const float4*>(src + int64_t(s0 + t) * 128 * bn))
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int t = 0; t < 6; ++t)
+                if (s0 + t < splits) { a[0] += v[t].x; a[1] += v[t].y; a[2] += v[t].z; a[3] += v[t].w; }
         }
         if (n + 4 <= N) {
             uint2 o;
