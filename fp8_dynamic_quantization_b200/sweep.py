@@ -5,8 +5,9 @@
     python -m fp8_dynamic_quantization_b200.sweep --op group128 --m 16384 --k 7168 --reps 3
 
 Every measurement is the median over `reps` of one call, timed with CUDA
-events on the launching stream.  Mode "cold": an L2 flush (a 256 MB write)
-and a ~100 us GPU sleep run before every call, outside the timed interval
+events on the launching stream.  Mode "cold": an L2 flush (a 256 MB read,
+which leaves only clean lines in L2) and a GPU sleep run before every call,
+outside the timed interval
 (the sleep hides the host's launch overhead).  Mode "graph":
 `reps` calls captured in one CUDA graph and replayed; time / reps (this is how
 the pages timed their amax kernel; inputs that fit in L2 stay L2-warm).
@@ -48,7 +49,10 @@ class Timer:
         torch.cuda.synchronize()
         ts = []
         for _ in range(reps):
-            self.flush_buf.fill_(1)
+            # evict the inputs by reading a buffer larger than L2: L2 is left
+            # holding clean lines, so the timed call does not also pay for
+            # writing back someone else's dirty data
+            self.flush_buf.max()
             # keep the GPU busy while the host prepares the call, so host-side
             # overhead never shows up between the two events
             torch.cuda._sleep(200_000)
