@@ -234,7 +234,9 @@ bool tile_override(TableRow* out) {
 // split along K into S = min(SMs / tail, K blocks / 2) ranges instead, so it
 // takes about 1/S of a tile time; tail_reduce_kernel then adds the S fp32
 // partials of each tail tile in fixed order.  ws_cap bounds the workspace
-// this may use (S shrinks to fit; below 2 the tail stays whole).
+// either split may use: split-K shrinks to fit (to 1, except where the
+// swapped kernel needs at least 2), the tail's S shrinks to fit (below 2 the
+// tail stays whole).
 GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = false,
                    size_t ws_cap = ~size_t(0)) {
     GemmPlan pl{};
@@ -262,6 +264,10 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
         splits = std::min(splits, std::max(1, G / 2));   // at least 2 K blocks per split
     }
     splits = std::max(1, std::min(splits, G));
+    if (splits > 1) {   // split-K partials must fit ws_cap: fewer splits if not
+        const size_t per_split = size_t(M) * size_t((N + 7) / 8 * 8) * sizeof(float);
+        splits = int(std::max<size_t>(1, std::min<size_t>(size_t(splits), ws_cap / per_split)));
+    }
     if (pl.swap) {   // the swapped kernel stages at most 64 K blocks of scales per unit
         while ((G + splits - 1) / splits > 64) ++splits;
     }
@@ -937,7 +943,8 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, cons
     DeviceInfo* d = nullptr;
     int rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
-    // regular split-K partials must fit the scratch; a split tail is cut to fit it
+    // the launch is planned to fit the scratch (fewer K splits); only a swapped
+    // skinny shape that needs 2+ splits larger than the scratch is refused
     if (plan_gemm(M, N, K, d->sms, false, kNoAllocScratchBytes).ws_bytes > kNoAllocScratchBytes)
         return FP8Q_ERR_WORKSPACE;
     void* scratch = nullptr;

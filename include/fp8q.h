@@ -311,14 +311,16 @@ int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa,
  * the workspace.  The split-K partial sums that fp8_block_gemm would put in
  * the caller's workspace go to a fixed scratch array inside the library
  * instead: FP8Q_NOALLOC_MAX_SCRATCH_BYTES (8 MiB) per device, reserved by
- * every device that loads the library until the process exits.  Shapes
- * whose launch needs more scratch than that (fp8_block_gemm_workspace_size
- * (M,N,K) > FP8Q_NOALLOC_MAX_SCRATCH_BYTES) are rejected with
- * FP8Q_ERR_WORKSPACE before anything is enqueued; use fp8_block_gemm for
- * them.  The one exception is a split last wave (see fp8_block_gemm): its
- * tiles are split into fewer K ranges when the scratch is too small for the
- * split fp8_block_gemm would use, so the bytes of those tiles can differ
- * from fp8_block_gemm's in rounding, within the same tolerance.
+ * every device that loads the library until the process exits.  The launch
+ * is planned to fit that scratch: where fp8_block_gemm would split K (or
+ * its last wave, see fp8_block_gemm) into more partial sums than the
+ * scratch holds, this call uses fewer K ranges, so its bytes can differ
+ * from fp8_block_gemm's in rounding, within the same tolerance.  A shape is
+ * rejected with FP8Q_ERR_WORKSPACE, before anything is enqueued, only when
+ * even the fewest K ranges its launch allows do not fit: skinny M (at most
+ * 32 rows, run with the operands swapped) with K > 8192 needs at least two
+ * ranges, 2 * M * N * 4 bytes (N rounded up to a multiple of 8).  Use
+ * fp8_block_gemm for those.
  *
  * The call allocates nothing: no cudaMalloc, cudaFree or allocating
  * library routine.  The first call on each device looks up the scratch
