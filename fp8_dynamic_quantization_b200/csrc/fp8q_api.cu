@@ -450,7 +450,20 @@ const char* fp8q_status_string(int status) {
     }
 }
 
-int fp8q_abi_version(void) { return (1 << 16) | 0; }
+int fp8q_abi_version(void) { return (1 << 16) | 1; }
+
+// Host only: the launch plan fp8_block_gemm (fp32, per-tensor and
+// per-channel scales) would use on a device with `sms` SMs.
+int fp8q_gemm_plan(int64_t M, int64_t N, int64_t K, int sms, size_t ws_cap, int* plan, size_t* ws_bytes) {
+    if (M <= 0 || N <= 0 || K <= 0 || sms <= 0 || !plan || !ws_bytes) return FP8Q_ERR_INVALID_ARG;
+    if (K % 128 || M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    const GemmPlan pl = plan_gemm(M, N, K, sms, false, ws_cap);
+    const int v[11] = {pl.swap ? 1 : 0, pl.pair ? 1 : 0, pl.bn, pl.stages, pl.splits, pl.tiles_p,
+                       pl.tiles_q, pl.units, pl.grid, pl.tail_tiles, pl.tail_splits};
+    for (int i = 0; i < 11; ++i) plan[i] = v[i];
+    *ws_bytes = pl.ws_bytes;
+    return FP8Q_OK;
+}
 
 // ------------------------------------------------------------ per-tensor
 size_t fp8_act_quant_per_tensor_workspace_size(int64_t, int64_t) {

@@ -342,6 +342,21 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa,
 /* Device status                                                       */
 /* ------------------------------------------------------------------ */
 
+/* The launch plan fp8_block_gemm, fp8_gemm_per_tensor and
+ * fp8_gemm_per_channel use for (M, N, K) on a device with `sms` SMs, with
+ * the split-K partials (or those of a split last wave) limited to ws_cap
+ * bytes (SIZE_MAX: no limit; fp8_block_gemm_noalloc plans with its
+ * scratch size).  Host only: no device is touched, so it runs anywhere.
+ * plan[0..10] receives: operands swapped (0/1), CTA pair (0/1), tile
+ * width BN, pipeline stages, K splits, tiles along the MMA's M operand,
+ * tiles along its N operand, work units, grid size, tail tiles split along
+ * K, K ranges per tail tile.  *ws_bytes receives the workspace the plan
+ * needs.  FP8Q_ERR_INVALID_ARG for non-positive sizes or null outputs,
+ * FP8Q_ERR_UNSUPPORTED_SHAPE for K % 128 != 0.  The pages have no
+ * counterpart: it exposes this library's launch selection for tests. */
+int fp8q_gemm_plan(int64_t M, int64_t N, int64_t K, int sms, size_t ws_cap,
+                   int* plan, size_t* ws_bytes);
+
 /* Synchronises the current device and stores in *status the first error a
  * kernel recorded since the last reset (FP8Q_OK if none; FP8Q_ERR_TIMEOUT
  * when a bounded wait gave up).  reset != 0 clears it afterwards. */

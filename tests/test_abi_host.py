@@ -150,3 +150,90 @@ def test_new_quant_argument_checks(cuda_lib, name):
     assert f(A, 4, 256, 256, B, 256, None, None) == INVALID
     assert f(A + 8, 4, 256, 256, B, 256, C, None) == MISALIGNED
     assert f(A, 0, 256, 256, B, 256, C, None) == OK                                # empty
+
+
+# ------------------------------------------------------------ launch plans
+PLAN_KEYS = ("swap", "pair", "bn", "stages", "splits", "tiles_p", "tiles_q", "units", "grid",
+             "tail_tiles", "tail_splits")
+NO_CAP = (1 << 64) - 1
+NOALLOC_CAP = 8 << 20
+
+
+def gemm_plan(lib, m, n, k, sms=148, cap=NO_CAP):
+    out = (ctypes.c_int * 11)()
+    ws = ctypes.c_size_t(0)
+    rc = lib.fp8q_gemm_plan(m, n, k, sms, cap, out, ctypes.byref(ws))
+    assert rc == OK
+    plan = dict(zip(PLAN_KEYS, list(out)))
+    plan["ws"] = ws.value
+    return plan
+
+
+def test_plan_argument_checks(cuda_lib):
+    out = (ctypes.c_int * 11)()
+    ws = ctypes.c_size_t(0)
+    assert cuda_lib.fp8q_gemm_plan(4, 4, 100, 148, NO_CAP, out, ctypes.byref(ws)) == SHAPE
+    assert cuda_lib.fp8q_gemm_plan(0, 4, 128, 148, NO_CAP, out, ctypes.byref(ws)) == INVALID
+    assert cuda_lib.fp8q_gemm_plan(4, 4, 128, 0, NO_CAP, out, ctypes.byref(ws)) == INVALID
+    assert cuda_lib.fp8q_gemm_plan(4, 4, 128, 148, NO_CAP, None, ctypes.byref(ws)) == INVALID
+
+
+def test_plan_prefill_tiles_and_split_last_wave(cuda_lib):
+    # 4096 x 7168: 32 x 28 = 896 tiles of 128 x 256 = 6 waves of 148 + 8;
+    # the 8 are split into min(148 // 8, 56 // 2) = 18 K ranges
+    p = gemm_plan(cuda_lib, 4096, 7168, 7168)
+    assert (p["swap"], p["pair"], p["bn"], p["splits"]) == (0, 0, 256, 1)
+    assert (p["tiles_p"], p["tiles_q"], p["tail_tiles"], p["tail_splits"]) == (32, 28, 8, 18)
+    assert p["units"] == 888 + 8 * 18 and p["grid"] == 148
+    assert p["ws"] == 8 * 18 * 128 * 256 * 4
+    # last waves of 84 and 112 tiles hold more than half the SMs: whole tiles
+    for n, tail in ((18432, 84), (24576, 112)):
+        p = gemm_plan(cuda_lib, 4096, n, 7168)
+        assert (p["tiles_p"] * p["tiles_q"]) % 148 == tail
+        assert (p["tail_tiles"], p["units"], p["ws"]) == (0, p["tiles_p"] * p["tiles_q"], 0)
+
+
+def test_plan_tile_choice_by_m_and_n(cuda_lib):
+    def key(m, n):
+        p = gemm_plan(cuda_lib, m, n, 7168)
+        return ("swap" if p["swap"] else "normal", p["bn"])
+    assert key(1, 18432) == ("swap", 16) and key(16, 7168) == ("swap", 16)
+    assert key(17, 2048) == ("swap", 32) and key(32, 18432) == ("swap", 32)
+    for m in (33, 64, 128):
+        assert key(m, 2048) == ("normal", 128)
+        assert key(m, 7168) == ("normal", 256)
+        assert key(m, 18432) == ("normal", 128)
+    for m in (129, 256, 512, 4096):
+        for n in (2048, 7168, 18432):
+            assert key(m, n) == ("normal", 256)
+
+
+def test_plan_split_k_fills_the_sms_and_respects_a_cap(cuda_lib):
+    # 64 x 7168: 1 x 28 tiles of 128 x 256 -> 148 // 28 = 5 K ranges
+    p = gemm_plan(cuda_lib, 64, 7168, 7168)
+    assert (p["splits"], p["units"]) == (5, 28 * 5)
+    assert p["ws"] == 5 * 64 * 7168 * 4
+    # with the no-alloc scratch as the cap: 8 MiB // (64 * 7168 * 4) = 4
+    q = gemm_plan(cuda_lib, 64, 7168, 7168, cap=NOALLOC_CAP)
+    assert (q["splits"], q["units"]) == (4, 28 * 4) and q["ws"] <= NOALLOC_CAP
+    # skinny M: 144 swapped weight tiles, too few K blocks to split further
+    p = gemm_plan(cuda_lib, 16, 18432, 7168)
+    assert (p["swap"], p["tiles_p"], p["tiles_q"], p["splits"], p["ws"]) == (1, 144, 1, 1, 0)
+
+
+def test_plan_cap_cuts_the_split_tail_and_the_swapped_minimum(cuda_lib):
+    # 4000 x 7100 x 4608: 896 tiles, tail of 8, 36 K blocks -> 18 ranges,
+    # 18 MiB of partials; under the 8 MiB cap 8 ranges
+    p = gemm_plan(cuda_lib, 4000, 7100, 4608)
+    assert (p["tail_tiles"], p["tail_splits"]) == (8, 18) and p["ws"] > NOALLOC_CAP
+    q = gemm_plan(cuda_lib, 4000, 7100, 4608, cap=NOALLOC_CAP)
+    assert (q["tail_tiles"], q["tail_splits"]) == (8, 8) and q["ws"] <= NOALLOC_CAP
+    # 32 swapped tokens with 65 K blocks need 2 K ranges whatever the cap
+    q = gemm_plan(cuda_lib, 32, 32776, 8320, cap=NOALLOC_CAP)
+    assert q["swap"] == 1 and q["splits"] == 2 and q["ws"] == 2 * 32 * 32776 * 4 > NOALLOC_CAP
+
+
+def test_plan_depends_on_the_sm_count(cuda_lib):
+    # 4096 x 7168 on 132 SMs: 896 = 6 * 132 + 104 -> more than half a wave
+    p = gemm_plan(cuda_lib, 4096, 7168, 7168, sms=132)
+    assert (p["tail_tiles"], p["grid"]) == (0, 132)
