@@ -116,45 +116,74 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def parse_clock_rows(text, t0=None, t1=None):
+    """Summary of nvidia-smi CSV rows (timestamp first, then ClockSampler's
+    fields): median SM clock, max clock, active throttle reasons.  Only rows
+    stamped inside [t0, t1] (host wall-clock seconds, the timed region) count
+    when t0/t1 are given and any row falls inside; otherwise all rows count."""
+    import datetime
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    rows = []
+    for line in text.strip().splitlines():
+        r = [c.strip() for c in line.split(",")]
+        if len(r) < 10:
+            continue
+        try:
+            ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            ts = None
+        rows.append((ts, r[1:]))
+    if not rows:
+        return None
+    inside = [r for ts, r in rows if t0 is not None and ts is not None and t0 <= ts <= t1]
+    use = inside if inside else [r for _, r in rows]
+    sm = [float(r[1]) for r in use if r[1].replace(".", "").isdigit()]
+    mx = [float(r[2]) for r in use if r[2].replace(".", "").isdigit()]
+    reasons = sorted({names[i] for r in use for i in range(4) if r[5 + i] == "Active"})
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+            "reasons": reasons, "samples": len(use), "in_timed_region": bool(inside)}
+
+
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 200 ms."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms; the summary
+    keeps the samples stamped inside the timed region."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.t0 = self.t1 = None
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "50"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
+        time.sleep(0.1)                      # first samples before the timed region
+
+    def mark(self, begin: bool):
+        """Host wall-clock bounds of the timed region."""
+        if begin:
+            self.t0 = time.time()
+        else:
+            self.t1 = time.time()
 
     def stop(self):
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             out, _ = self.proc.communicate(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
             out, _ = self.proc.communicate()
-        rows = [r.split(", ") for r in out.strip().splitlines() if r.strip()]
-        rows = [r for r in rows if len(r) >= 9]
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].strip() == "Active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        return parse_clock_rows(out, self.t0, self.t1)
 
 
 def host_cores():
@@ -278,11 +307,13 @@ def our_arm(args, rank, world, local_rank):
     torch.cuda.synchronize(dev)
     clocks.start()
     launches0 = lib.fp8q_launch_count()
+    clocks.mark(True)
     start.record(stream)
     for s in range(args.steps):
         step(events[s])
     end.record(stream)
     torch.cuda.synchronize(dev)
+    clocks.mark(False)
     launches = lib.fp8q_launch_count() - launches0
     clk = clocks.stop()
     if dist is not None:
