@@ -399,6 +399,65 @@ def test_f64_to_bf16_matches_torch(oracle_mod):
     np.testing.assert_array_equal(ours, ref)
 
 
+def _bf16_rne_exact(v: float) -> int:
+    """bf16 bit pattern of the float64 value v rounded once, to nearest with
+    ties to even, computed with exact rationals: the float64 value as a
+    Fraction, its bf16 quantum (8 significant bits, normal range from
+    2^-126, subnormal quantum 2^-133), round(n) on the exact quotient
+    (Python rounds a Fraction half to even), overflow to infinity."""
+    import math
+    import struct
+    from fractions import Fraction
+    sign = 0x8000 if math.copysign(1.0, v) < 0 else 0
+    a = Fraction(abs(v))
+    if a == 0:
+        return sign
+    k = math.frexp(abs(v))[1] - 1                  # floor(log2 |v|)
+    quantum = Fraction(2) ** (max(k, -126) - 7)
+    r = round(a / quantum) * quantum
+    if r >= Fraction(2) ** 128:
+        return sign | 0x7F80
+    return sign | (struct.unpack("<I", struct.pack("<f", float(r)))[0] >> 16)
+
+
+def _bf16_value(bits: int) -> float:
+    import struct
+    return struct.unpack("<f", struct.pack("<I", bits << 16))[0]
+
+
+def test_f64_to_bf16_rounds_float64_values_once(oracle_mod):
+    """Float64 values that fp32 cannot hold: the exact midpoints between
+    neighbouring bf16 values, one float64 ulp either side of them, values a
+    hair above a midpoint whose fp32 rounding lands on the midpoint (rounding
+    through fp32 first would then tie to even and go the wrong way),
+    subnormal and overflow boundaries, and random full-precision values --
+    against a one-rounding reference built from exact rationals.  A
+    double-rounding variant (float64 -> fp32 -> bf16) is checked to fail on
+    these cases, so the pin would catch that mistake."""
+    import math
+    g = np.random.default_rng(11)
+    vals = []
+    lo_bits = g.integers(0x0001, 0x7F7F, 400)                      # finite, nonzero bf16
+    for b in list(lo_bits) + [0x0001, 0x007F, 0x0080, 0x3F80, 0x7F7E]:
+        lo, hi = _bf16_value(int(b)), _bf16_value(int(b) + 1)
+        mid = (lo + hi) / 2.0                                        # exact in float64
+        vals += [mid, math.nextafter(mid, math.inf), math.nextafter(mid, -math.inf)]
+        # just above the midpoint by less than half an fp32 ulp of it
+        vals.append(mid + math.ulp(mid) * 64.0)
+        vals.append(mid - math.ulp(mid) * 64.0)
+    top = _bf16_value(0x7F7F)
+    vals += [top + math.ulp(top) * (2.0 ** 44), 2.0 ** 128 - 2.0 ** 119,
+             math.nextafter(2.0 ** 128 - 2.0 ** 119, 0.0), 2.0 ** -134, math.nextafter(2.0 ** -134, 1.0),
+             5e-324, 1e-300, 3 * 2.0 ** -135]
+    vals += list(g.standard_normal(2000) * 2.0 ** g.integers(-140, 128, 2000).astype(np.float64))
+    vals = np.array([v for x in vals for v in (x, -x)], dtype=np.float64)
+    ours = oracle_mod.f64_to_bf16(vals)
+    exact = np.array([_bf16_rne_exact(float(v)) for v in vals], dtype=np.uint16)
+    np.testing.assert_array_equal(ours, exact)
+    twice = torch.from_numpy(vals.astype(np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.count_nonzero(twice != exact) > 100, "the cases do not separate one rounding from two"
+
+
 def test_tolerance_formula(oracle_mod):
     tol = oracle_mod.gemm_tolerance(np.array([1.0, 1.5, -3.0, 0.0]), np.zeros(4))
     np.testing.assert_array_equal(tol, [2 * 2.0 ** -7, 2 * 2.0 ** -7, 2 * 2.0 ** -6, 2 * 2.0 ** -133])
