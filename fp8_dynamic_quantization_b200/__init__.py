@@ -28,7 +28,7 @@ __all__ = [
     "block_gemm_ue8m0", "linear_ue8m0", "act_quant_per_channel", "gemm_per_channel",
     "linear_per_channel",
     "block_gemm", "linear", "linear_fused", "gemm_per_tensor", "linear_per_tensor",
-    "device_status",
+    "device_status", "stream_status",
     "per_tensor_sharded", "Fp8qError", "library",
 ]
 
@@ -370,11 +370,22 @@ def linear(x: torch.Tensor, qb: torch.Tensor, sb: torch.Tensor) -> torch.Tensor:
 
 
 def device_status(reset: bool = True) -> int:
-    """Synchronise and return the first device-side error recorded by a
-    kernel (0 = none; 6 = a bounded wait timed out)."""
+    """Synchronise the device and return the first device-side error
+    recorded by a kernel on any stream (0 = none; 6 = a bounded wait timed
+    out)."""
     lib = _abi.load()
     v = ctypes.c_int(0)
     _abi.check(lib.fp8q_device_status(ctypes.byref(v), int(reset)), "fp8q_device_status")
+    return v.value
+
+
+def stream_status(stream: torch.cuda.Stream | None = None) -> int:
+    """Wait for `stream` (default: the current stream) only, then return and
+    clear the first device-side error its kernels recorded (0 = none)."""
+    lib = _abi.load()
+    st = stream if stream is not None else torch.cuda.current_stream()
+    v = ctypes.c_int(0)
+    _abi.check(lib.fp8q_get_last_device_status(st.cuda_stream, ctypes.byref(v)), "fp8q_get_last_device_status")
     return v.value
 
 

@@ -41,7 +41,9 @@ SIGNATURES = {
     "fp8_block_gemm_ue8m0": (_int, [_p, _i64, _p, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p, _sz, _p]),
     "fp8_block_gemm_noalloc": (_int, [_p, _i64, _p, _p, _i64, _p, _p, _i64, _i64, _i64, _i64, _p]),
     "fp8q_gemm_plan": (_int, [_i64, _i64, _i64, _int, _sz, _p, _p]),
+    "fp8q_get_last_device_status": (_int, [_p, _p]),
     "fp8q_device_status": (_int, [_p, _int]),
+    "fp8q_set_wait_budget_cycles": (ctypes.c_longlong, [ctypes.c_longlong]),
     "fp8q_launch_count": (ctypes.c_ulonglong, []),
 }
 

@@ -41,6 +41,7 @@ struct DeviceInfo {
     bool ready = false;
     int status = FP8Q_OK;
     int sms = 0;
+    int index = 0;
 };
 
 constexpr int kMaxDevices = 64;
@@ -77,6 +78,7 @@ int device_info(DeviceInfo** out) {
                 return FP8Q_ERR_NO_DEVICE;
             }
             d.status = FP8Q_OK;
+            d.index = dev;
             if (prop.major != 10) d.status = FP8Q_ERR_NO_DEVICE;
             d.sms = prop.multiProcessorCount;
             if (d.status == FP8Q_OK) {
@@ -126,6 +128,36 @@ int device_info(DeviceInfo** out) {
     }
     *out = &d;
     return d.status;
+}
+
+// Stream -> error-word slot (g_stream_status), per device.  Slots 1.. are
+// handed out in the order streams first ask for one; once they are all
+// taken, later streams share slot 0.  A stream handle that CUDA recycles
+// for a new stream keeps the slot.
+cudaStream_t g_slot_stream[kMaxDevices][kStatusSlots];
+int g_slots_used[kMaxDevices];
+std::mutex g_slot_mutex;
+
+int status_slot(int dev, cudaStream_t st) {
+    thread_local int last_dev = -1, last_slot = 0;
+    thread_local cudaStream_t last_st = nullptr;
+    if (dev == last_dev && st == last_st) return last_slot;
+    int slot = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_slot_mutex);
+        const int n = g_slots_used[dev];
+        for (int i = 1; i <= n && slot == 0; ++i)
+            if (g_slot_stream[dev][i] == st) slot = i;
+        if (slot == 0 && n + 1 < kStatusSlots) {
+            slot = n + 1;
+            g_slot_stream[dev][slot] = st;
+            g_slots_used[dev] = slot;
+        }
+    }
+    last_dev = dev;
+    last_st = st;
+    last_slot = slot;
+    return slot;
 }
 
 std::atomic<unsigned long long> g_launches{0};
@@ -186,7 +218,11 @@ bool per_tensor_two_pass_forced() {
 // Bound on every barrier wait inside the GEMM, in SM clock cycles (about
 // two seconds by default).  FP8Q_WAIT_BUDGET_CYCLES overrides it for fault
 // testing; it never changes the result of a call that completes.
+std::atomic<long long> g_wait_budget_override{-1};
+
 long long wait_budget_cycles() {
+    const long long o = g_wait_budget_override.load(std::memory_order_relaxed);
+    if (o >= 0) return o;
     static const long long v = [] {
         const char* e = std::getenv("FP8Q_WAIT_BUDGET_CYCLES");
         if (e && e[0]) {
@@ -699,6 +735,29 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 
 }  // extern "C"
 
+// Host-side argument checks shared by every GEMM entry point, run before
+// anything touches the device, in this order: negative sizes, unsupported
+// shapes (K % 128, sizes beyond INT_MAX), empty products (FP8Q_OK with
+// *empty set: nothing to do), null pointers, leading dimensions, alignment.
+// mode as in run_gemm.
+static int check_gemm_args(int mode, const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb,
+                           int64_t ldb, const float* sb, const void* y, int64_t ldy, int64_t M, int64_t N,
+                           int64_t K, const uint16_t* x, int64_t ldx, bool* empty) {
+    const bool ue8m0 = mode == 2, fused = mode == 4;
+    *empty = false;
+    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
+    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) { *empty = true; return FP8Q_OK; }
+    if ((fused ? !x : (!qa || !sa)) || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+    if ((fused ? ldx < K : lda < K) || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+    if ((fused ? (!aligned16(x) || ldx % 8) : (!aligned16(qa) || lda % 16)) ||
+        !aligned16(qb) || !aligned16(y) || ldb % 16 || (ldy * 2) % 16 ||
+        (!ue8m0 && ((!fused && !aligned4(sa)) || !aligned4(sb))))
+        return FP8Q_ERR_MISALIGNED;
+    return FP8Q_OK;
+}
+
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                     void* workspace, size_t workspace_bytes, void* stream, int mode,
@@ -706,21 +765,14 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
                     size_t ws_cap = ~size_t(0)) {
     // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes;
     // 3: per-channel fp32 scales; 4: fp32 block scales with the group-128
-    // quantisation of bf16 tokens x fused in (swapped tiles of <= 64 tokens;
+    // quantisation of bf16 tokens x fused in (swapped tiles of <= 32 tokens;
     // qa and sa unused)
     const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3, fused = mode == 4;
-    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
-    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
-    if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
-    if (M == 0 || N == 0) return FP8Q_OK;
-    if ((fused ? !x : (!qa || !sa)) || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
-    if ((fused ? ldx < K : lda < K) || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
-    if ((fused ? (!aligned16(x) || ldx % 8) : (!aligned16(qa) || lda % 16)) ||
-        !aligned16(qb) || !aligned16(y) || ldb % 16 || (ldy * 2) % 16 ||
-        (!ue8m0 && ((!fused && !aligned4(sa)) || !aligned4(sb))))
-        return FP8Q_ERR_MISALIGNED;
+    bool empty = false;
+    int rc = check_gemm_args(mode, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, x, ldx, &empty);
+    if (rc != FP8Q_OK || empty) return rc;
     DeviceInfo* d = nullptr;
-    int rc = device_info(&d);
+    rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (K == 0) {
@@ -770,6 +822,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return FP8Q_ERR_CUDA;
     if (fused && !make_x_tmap(&tsa, x, M, K, ldx, pl.bn)) return FP8Q_ERR_CUDA;   // the token tiles
     p.wait_budget = wait_budget_cycles();
+    p.status_slot = uint8_t(status_slot(d->index, st));
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d"
                              " tail=%dx%d\n",
@@ -949,12 +1002,13 @@ int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa, cons
 int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb,
                            int64_t ldb, const float* sb, void* y, int64_t ldy, int64_t M, int64_t N,
                            int64_t K, void* stream) {
-    // Shape/pointer errors are reported exactly as fp8_block_gemm reports them.
-    if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
-    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
-    if (M == 0 || N == 0) return FP8Q_OK;
+    // Argument errors first, with fp8_block_gemm's checks and codes, before
+    // the device is queried or the launch is planned against the scratch.
+    bool empty = false;
+    int rc = check_gemm_args(0, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, nullptr, 0, &empty);
+    if (rc != FP8Q_OK || empty) return rc;
     DeviceInfo* d = nullptr;
-    int rc = device_info(&d);
+    rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
     // the launch is planned to fit the scratch (fewer K splits); only a swapped
     // skinny shape that needs 2+ splits larger than the scratch is refused
@@ -978,13 +1032,44 @@ int fp8q_device_status(int* status, int reset) {
     int rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
     if (cudaDeviceSynchronize() != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
-    *status = v;
+    int v[kStatusSlots];
+    if (cudaMemcpyFromSymbol(v, g_stream_status, sizeof(v)) != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
+    *status = FP8Q_OK;
+    for (int i = 0; i < kStatusSlots && *status == FP8Q_OK; ++i) *status = v[i];
     if (reset) {
-        const int z = 0;
-        if (cudaMemcpyToSymbol(g_device_status, &z, sizeof(int)) != cudaSuccess) return FP8Q_ERR_CUDA;
+        std::memset(v, 0, sizeof(v));
+        if (cudaMemcpyToSymbol(g_stream_status, v, sizeof(v)) != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
     }
+    return FP8Q_OK;
+}
+
+long long fp8q_set_wait_budget_cycles(long long cycles) {
+    const long long prev = wait_budget_cycles();
+    g_wait_budget_override.store(cycles < 0 ? -1 : cycles, std::memory_order_relaxed);
+    return prev;
+}
+
+int fp8q_get_last_device_status(void* stream, int* status) {
+    if (!status) return FP8Q_ERR_INVALID_ARG;
+    DeviceInfo* d = nullptr;
+    int rc = device_info(&d);
+    if (rc != FP8Q_OK) return rc;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t off = size_t(status_slot(d->index, st)) * sizeof(int);
+    int v = 0;
+    const int z = 0;
+    // the copies are ordered after this stream's kernels; only this stream waits
+    if (cudaMemcpyFromSymbolAsync(&v, g_stream_status, sizeof(int), off, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+        cudaGetLastError();
+        return FP8Q_ERR_CUDA;
+    }
+    if (v != 0 && (cudaMemcpyToSymbolAsync(g_stream_status, &z, sizeof(int), off, cudaMemcpyHostToDevice, st) != cudaSuccess ||
+                   cudaStreamSynchronize(st) != cudaSuccess)) {
+        cudaGetLastError();
+        return FP8Q_ERR_CUDA;
+    }
+    *status = v;
     return FP8Q_OK;
 }
 

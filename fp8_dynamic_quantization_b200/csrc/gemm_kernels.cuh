@@ -105,6 +105,7 @@ struct GemmParams {
     uint8_t scale_vec4;  // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
     uint8_t sf_words;    // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
     uint8_t pdl;         // launched as a programmatic dependent of the kernel producing A and sa
+    uint8_t status_slot; // error word of the launching stream (g_stream_status index)
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 static_assert(sizeof(GemmParams) <= 104, "GemmParams size");
@@ -388,7 +389,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
 
-    auto fail = [&]() { *abort_flag = 1; record_error(6 /* FP8Q_ERR_TIMEOUT */); };
+    auto fail = [&]() { *abort_flag = 1; record_error(p.status_slot, 6 /* FP8Q_ERR_TIMEOUT */); };
 
     // ------------------------------------------ token quantiser (fused mode)
     // Run by warps 2 and 3; `mine` is this warp's index among them.

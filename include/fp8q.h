@@ -54,8 +54,9 @@
  *     FP8Q_PER_TENSOR_PATH=twopass the two-pass per-tensor path (measurement);
  *     FP8Q_LINEAR=fused|serial how fp8_linear_group128 runs (measurement);
  *     FP8Q_WAIT_BUDGET_CYCLES bounds the GEMM's device-side waits (fault
- *     testing); both are read once per process.  No environment variable
- *     changes the result of a call that completes.
+ *     testing; fp8q_set_wait_budget_cycles changes it at run time); these
+ *     are read once per process.  No environment variable changes the
+ *     result of a call that completes.
  */
 #ifndef FP8Q_H
 #define FP8Q_H
@@ -248,8 +249,9 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * fills at most half the SMs, the tiles of that wave are split along K and
  * their fp32 partials are added in fixed order by a second kernel (the
  * call then enqueues two kernels); results are deterministic for a given
- * shape and device.  Bounded device waits report FP8Q_ERR_TIMEOUT through
- * fp8q_device_status. */
+ * shape and device.  A bounded device wait that gives up records
+ * FP8Q_ERR_TIMEOUT in the error word of `stream`, read by
+ * fp8q_get_last_device_status (or fp8q_device_status for every stream). */
 int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                    const uint8_t* qb, int64_t ldb, const float* sb,
                    void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
@@ -325,7 +327,13 @@ int fp8_block_gemm_ue8m0(const uint8_t* qa, int64_t lda, const uint8_t* sa,
  * The call allocates nothing: no cudaMalloc, cudaFree or allocating
  * library routine.  The first call on each device looks up the scratch
  * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture begins.
+ * make that first call before any stream capture begins.  The scratch is
+ * part of the library's device code, which CUDA loads onto a device when
+ * a call first touches the library there (lazy module loading); that load
+ * claims the 8 MiB.  A process that reserves the whole device pool at
+ * start-up must therefore make its first fp8_block_gemm_noalloc call (with
+ * real operands) or one fp8q_device_status call on each device before it
+ * reserves the pool, as it must before any stream capture.
  *
  * All calls on a device share the one scratch array, which keeps the last
  * call's contents; each call overwrites every partial sum it reads, so no
@@ -357,10 +365,33 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa,
 int fp8q_gemm_plan(int64_t M, int64_t N, int64_t K, int sms, size_t ws_cap,
                    int* plan, size_t* ws_bytes);
 
-/* Synchronises the current device and stores in *status the first error a
- * kernel recorded since the last reset (FP8Q_OK if none; FP8Q_ERR_TIMEOUT
- * when a bounded wait gave up).  reset != 0 clears it afterwards. */
+/* Device-side errors.  A kernel that meets an error it cannot report
+ * through its return value (a bounded wait that gave up: FP8Q_ERR_TIMEOUT)
+ * records it in the error word of the stream it was launched on, and the
+ * first error recorded stays until it is read and cleared.  Streams get
+ * their own word in the order they first use one (255 per device); streams
+ * beyond that share one word.  The pages have no counterpart: they define
+ * no device-side failure. */
+
+/* Waits for the work enqueued on `stream` (only that stream: it does not
+ * synchronise the device), then stores in *status the first error a kernel
+ * launched on it recorded since the last read (FP8Q_OK if none), and clears
+ * it.  FP8Q_ERR_INVALID_ARG for a null status, FP8Q_ERR_CUDA if the stream
+ * failed. */
+int fp8q_get_last_device_status(void* stream, int* status);
+
+/* Synchronises the current device and stores in *status the first error
+ * recorded on any stream of it since the last reset (FP8Q_OK if none).
+ * reset != 0 clears every stream's word afterwards. */
 int fp8q_device_status(int* status, int reset);
+
+/* Sets the bound on every device-side wait of the GEMM kernels launched
+ * from now on, in SM clock cycles (default about two seconds, or
+ * FP8Q_WAIT_BUDGET_CYCLES); a negative value restores the default.
+ * Returns the bound in force before the call.  For fault testing: a bound
+ * of 0 makes the first wait that is not already satisfied give up.  It
+ * never changes the result of a call that completes. */
+long long fp8q_set_wait_budget_cycles(long long cycles);
 
 /* Number of kernels this library has launched in the process so far (all
  * devices, all streams); a diagnostic for benchmarks. */

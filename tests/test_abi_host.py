@@ -19,7 +19,7 @@ D = 0x40000
 
 def declared_functions():
     text = open(HEADER).read()
-    return re.findall(r"^(?:const char\*|int|size_t|unsigned long long)\s+(\w+)\s*\(", text, re.M)
+    return re.findall(r"^(?:const char\*|int|size_t|unsigned long long|long long)\s+(\w+)\s*\(", text, re.M)
 
 
 def test_header_declares_the_abi():
@@ -84,8 +84,21 @@ def test_block128_argument_checks(cuda_lib):
     assert f(A, 200, 256, 256, B + 4, 256, C, None) == MISALIGNED
 
 
-def test_gemm_argument_checks(cuda_lib):
-    f = cuda_lib.fp8_block_gemm
+def _gemm_entry(cuda_lib, name):
+    """fp8_block_gemm, or fp8_block_gemm_noalloc behind the same argument
+    list (its workspace arguments dropped)."""
+    if name == "fp8_block_gemm":
+        return cuda_lib.fp8_block_gemm
+    g = cuda_lib.fp8_block_gemm_noalloc
+    return lambda qa, lda, sa, qb, ldb, sb, y, ldy, m, n, k, ws, wsb, st: g(qa, lda, sa, qb, ldb, sb, y, ldy,
+                                                                           m, n, k, st)
+
+
+@pytest.mark.parametrize("name", ["fp8_block_gemm", "fp8_block_gemm_noalloc"])
+def test_gemm_argument_checks(cuda_lib, name):
+    """Both GEMM entry points report argument errors with the same codes,
+    before they look for a device (this host has none) or plan a launch."""
+    f = _gemm_entry(cuda_lib, name)
     assert f(A, 200, B, C, 200, D, A, 64, 16, 64, 200, None, 0, None) == SHAPE     # K % 128
     assert f(A, 256, B, C, 256, D, A, 64, -1, 64, 256, None, 0, None) == INVALID
     assert f(A, 256, B, C, 256, D, A, 64, 0, 64, 256, None, 0, None) == OK          # empty M
@@ -97,6 +110,14 @@ def test_gemm_argument_checks(cuda_lib):
     assert f(A, 264, B, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == MISALIGNED  # lda pitch
     assert f(A, 256, B, C, 256, D, A, 60, 16, 60, 256, None, 0, None) == MISALIGNED  # ldy pitch
     assert f(A, 256, B + 1, C, 256, D, A, 64, 16, 64, 256, None, 0, None) == MISALIGNED
+    # a skinny shape beyond the no-alloc scratch (32 x 32776 x 8320) with a
+    # null output: the pointer error wins over any workspace question
+    assert f(A, 8320, B, C, 8320, D, None, 32776, 32, 32776, 8320, None, 0, None) == INVALID
+    # sizes beyond INT_MAX: unsupported, before any launch plan is made
+    big = 1 << 31
+    assert f(A, 256, B, C, 256, D, A, big, 16, big, 256, None, 0, None) == SHAPE
+    assert f(A, 256, B, C, 256, D, A, 64, big, 64, 256, None, 0, None) == SHAPE
+    assert f(A, big * 128, B, C, big * 128, D, A, 64, 16, 64, big * 128, None, 0, None) == SHAPE
 
 
 def test_no_device_status_without_gpu(cuda_lib):
@@ -107,6 +128,10 @@ def test_no_device_status_without_gpu(cuda_lib):
     assert f(A, 4, 128, 128, B, 128, C, None) == NO_DEVICE
     v = ctypes.c_int(0)
     assert cuda_lib.fp8q_device_status(ctypes.byref(v), 0) == NO_DEVICE
+    assert cuda_lib.fp8q_get_last_device_status(None, ctypes.byref(v)) == NO_DEVICE
+    assert cuda_lib.fp8q_get_last_device_status(None, None) == INVALID
+    # valid arguments: the no-alloc GEMM gets as far as looking for a device
+    assert cuda_lib.fp8_block_gemm_noalloc(A, 256, B, C, 256, D, A, 64, 16, 64, 256, None) == NO_DEVICE
     assert cuda_lib.fp8_block_gemm_workspace_size(16, 64, 256) == 0
 
 

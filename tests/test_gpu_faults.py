@@ -1,8 +1,9 @@
 """Failure detection without a GPU fault.
 
 A device-side wait that runs out must end the kernel with FP8Q_ERR_TIMEOUT in
-the library's status word (read by fp8q_device_status), write no outputs and
-leave the context usable.  The GEMM's barrier waits are bounded in SM clock
+the error word of the stream it was launched on (read by
+fp8q_get_last_device_status, or fp8q_device_status for all streams), write no
+outputs and leave the context usable.  The GEMM's barrier waits are bounded in SM clock
 cycles; FP8Q_WAIT_BUDGET_CYCLES=0 (read once per process, hence a child
 process) makes the first wait that is not already satisfied -- the MMA
 warp's wait for the first operand tile -- run out.  The kernel then stops
@@ -45,5 +46,48 @@ print("ok")
 def test_gemm_wait_timeout_is_reported(gpu, cuda_lib, oracle_mod):
     env = dict(os.environ, FP8Q_WAIT_BUDGET_CYCLES="0")
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
+CHILD_STREAMS = r'''
+import ctypes, sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import oracle
+import fp8_dynamic_quantization_b200 as fq
+from fp8_dynamic_quantization_b200 import _abi, inputs
+lib = _abi.load()
+dev = torch.device("cuda:0")
+fq.device_status(reset=True)
+qa, sa, qb, sb = inputs.gemm_operands(256, 1024, 1024, seed=7)
+ops = [torch.from_numpy(a).to(dev) for a in (qa, sa, qb, sb)]
+torch.cuda.synchronize()
+sa_, sb_ = torch.cuda.Stream(), torch.cuda.Stream()
+ya = torch.full((256, 1024), 3.0, dtype=torch.bfloat16, device=dev)
+yb = torch.full((256, 1024), 3.0, dtype=torch.bfloat16, device=dev)
+lib.fp8q_set_wait_budget_cycles(0)               # stream A's GEMM gives up at its first wait
+with torch.cuda.stream(sa_):
+    fq.block_gemm(*ops, out=ya)
+lib.fp8q_set_wait_budget_cycles(-1)              # the default bound again
+with torch.cuda.stream(sb_):
+    fq.block_gemm(*ops, out=yb)
+assert fq.stream_status(sb_) == 0, "stream B saw stream A's timeout"
+assert fq.stream_status(sa_) == 6, "expected FP8Q_ERR_TIMEOUT on stream A"
+assert fq.stream_status(sa_) == 0, "reading the status clears it"
+assert fq.device_status(reset=True) == 0
+assert bool(torch.all(ya == 3.0)), "the timed-out GEMM wrote output"
+R, T = oracle.block_gemm(qa, sa, qb, sb)
+err = np.abs(yb.float().cpu().numpy().astype(np.float64) - R)
+assert np.all(err <= oracle.gemm_tolerance(R, T)), "stream B's GEMM is wrong"
+print("ok")
+'''
+
+
+def test_timeout_is_reported_on_its_own_stream(gpu, cuda_lib, oracle_mod):
+    """A GEMM on stream A whose waits run out (bound 0) records
+    FP8Q_ERR_TIMEOUT in A's error word only: a GEMM launched right after on
+    stream B completes correctly, B's status reads FP8Q_OK without waiting
+    for A, and reading A's status clears it."""
+    r = subprocess.run([sys.executable, "-c", CHILD_STREAMS, ROOT], capture_output=True, text=True,
                        timeout=600)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
