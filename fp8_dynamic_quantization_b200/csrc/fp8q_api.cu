@@ -53,6 +53,48 @@ constexpr int kStreamU = 4;         // vectors per thread per iteration elsewher
 constexpr int kMaxPartials = 4096;  // per-tensor workspace partial slots
 constexpr int kBlocksPerSm = 8;     // 256-thread CTAs per SM for streaming kernels
 
+// Programmatic dependent launch of every kernel (the kernels' side is
+// pdl_begin / griddepcontrol in the device code): a launch may begin while
+// the previous kernel on the stream finishes, and waits for it before it
+// touches global memory.  FP8Q_PDL=0 launches without the attribute
+// (measurement; same results).
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = std::getenv("FP8Q_PDL");
+        return !(e && e[0] == '0');
+    }();
+    return on;
+}
+
+// cudaLaunchKernelEx with the programmatic-serialisation attribute and, for
+// cluster > 1, a 1-D cluster of that many CTAs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                   unsigned cluster, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = cluster;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 cudaError_t set_gemm_smem() {
     return cudaFuncSetAttribute(block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>,
@@ -100,8 +142,6 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
-                if (e == cudaSuccess) e = set_gemm_smem<16, true, 8, false, 4>();
-                if (e == cudaSuccess) e = set_gemm_smem<32, true, 7, false, 4>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 1>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true, 1>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 3>();
@@ -380,60 +420,13 @@ bool make_scale_tmap(CUtensorMap* m, const float* base, int64_t rows, int64_t G,
                CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Map of bf16 tokens x [rows, K] (row pitch ldx elements, a multiple of 8):
-// boxes of one 128-wide K block x box_rows rows, no swizzle; rows past the
-// end read as zero.
-bool make_x_tmap(CUtensorMap* m, const uint16_t* base, int64_t rows, int64_t K, int64_t ldx, int box_rows) {
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return false;
-    cuuint64_t dims[2] = {cuuint64_t(K), cuuint64_t(rows)};
-    cuuint64_t strides[1] = {cuuint64_t(ldx) * 2};
-    cuuint32_t box[2] = {128u, cuuint32_t(box_rows)};
-    cuuint32_t estr[2] = {1u, 1u};
-    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 // tsa/tsb: scale maps (staged-scale variants only; the others ignore them)
 template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& tsa, const CUtensorMap& tsb,
                  const GemmParams& p, int grid, cudaStream_t st) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
-    if (!PAIR && p.pdl) {
-        // programmatic dependent launch: may start while the previous kernel
-        // in the stream runs; the kernel waits for it before reading A or sa
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(unsigned(grid));
-        cfg.blockDim = dim3(C::kThreads);
-        cfg.dynamicSmemBytes = C::kSmemBytes;
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[0].val.programmaticStreamSerializationAllowed = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, tp, tq, tsa, tsb, p);
-        return;
-    }
-    if (!PAIR) {
-        block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS><<<grid, C::kThreads, C::kSmemBytes, st>>>(
-            tp, tq, tsa, tsb, p);
-        return;
-    }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(unsigned(grid));
-    cfg.blockDim = dim3(C::kThreads);
-    cfg.dynamicSmemBytes = C::kSmemBytes;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, tp, tq, tsa, tsb, p);
+    launch(block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, dim3(unsigned(grid)), dim3(C::kThreads),
+           C::kSmemBytes, st, PAIR ? 2u : 1u, tp, tq, tsa, tsb, p);
 }
 
 // ------------------------------------------------------------------ no-alloc GEMM scratch
@@ -539,23 +532,12 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
         if (log_enabled())
             std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: one cluster of %lld CTAs\n",
                          (long long)M, (long long)K, (long long)csize);
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(unsigned(csize));
-        cfg.blockDim = dim3(kClusterThreads);
-        cfg.stream = st;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = unsigned(csize);
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = csize > 1 ? 1 : 0;        // one CTA: a plain launch
         const uint16_t* xs = static_cast<const uint16_t*>(x);
         const cudaError_t e =
-            contig ? cudaLaunchKernelEx(&cfg, per_tensor_cluster_kernel<kClusterU, true, kClusterThreads>, xs,
-                                        nvec, vpr, ldx, q, ldq, scale)
-                   : cudaLaunchKernelEx(&cfg, per_tensor_cluster_kernel<kClusterU, false, kClusterThreads>, xs,
-                                        nvec, vpr, ldx, q, ldq, scale);
+            contig ? launch(per_tensor_cluster_kernel<kClusterU, true, kClusterThreads>, dim3(unsigned(csize)),
+                            dim3(kClusterThreads), 0, st, unsigned(csize), xs, nvec, vpr, ldx, q, ldq, scale)
+                   : launch(per_tensor_cluster_kernel<kClusterU, false, kClusterThreads>, dim3(unsigned(csize)),
+                            dim3(kClusterThreads), 0, st, unsigned(csize), xs, nvec, vpr, ldx, q, ldq, scale);
         if (e != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
         return launch_status(1);
     }
@@ -566,12 +548,12 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
                      (long long)M, (long long)K, grid);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (contig) {
-        amax_partial_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
-        apply_kernel<kStreamU, true, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials,
+        launch(amax_partial_kernel<kStreamU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
+        launch(apply_kernel<kStreamU, true, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials,
                                                                             grid, q, ldq, scale);
     } else {
-        amax_partial_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
-        apply_kernel<kStreamU, false, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials,
+        launch(amax_partial_kernel<kStreamU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
+        launch(apply_kernel<kStreamU, false, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials,
                                                                              grid, q, ldq, scale);
     }
     return launch_status(2);
@@ -600,11 +582,11 @@ int fp8_act_amax(const void* x, int64_t M, int64_t K, int64_t ldx, uint32_t* ama
     uint32_t* partials = static_cast<uint32_t*>(workspace);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (ldx == K)
-        amax_partial_kernel<kStreamU, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+        launch(amax_partial_kernel<kStreamU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
     else
-        amax_partial_kernel<kStreamU, false><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, partials);
+        launch(amax_partial_kernel<kStreamU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
     // Fold the partials into one word: a single CTA over `grid` words.
-    reduce_partials_kernel<<<1, kQuantThreads, 0, st>>>(partials, grid, amax_bits);
+    launch(reduce_partials_kernel, dim3(1), dim3(kQuantThreads), 0, st, 1u, partials, grid, amax_bits);
     return launch_status(2);
 }
 
@@ -620,16 +602,16 @@ int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t vpr = K / 8, nvec = M * vpr;
     if (nvec == 0) {
-        if (scale) scale_only_kernel<<<1, 32, 0, st>>>(amax_bits, scale);
+        if (scale) launch(scale_only_kernel, dim3(1), dim3(32), 0, st, 1u, amax_bits, scale);
         return launch_status();
     }
     const int grid = stream_grid(nvec, d->sms);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     if (ldx == K && ldq == K)
-        apply_kernel<kStreamU, true, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+        launch(apply_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, amax_bits, 1,
                                                                            q, ldq, scale);
     else
-        apply_kernel<kStreamU, false, true><<<grid, kQuantThreads, 0, st>>>(xs, nvec, vpr, ldx, amax_bits, 1,
+        launch(apply_kernel<kStreamU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, amax_bits, 1,
                                                                             q, ldq, scale);
     return launch_status();
 }
@@ -657,13 +639,13 @@ static int run_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     const bool contig = ldx == K && ldq == K;
     if (e8 && contig)
-        group128_quant_kernel<kGroupU, true, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        launch(group128_quant_kernel<kGroupU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     else if (e8)
-        group128_quant_kernel<kGroupU, false, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        launch(group128_quant_kernel<kGroupU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     else if (contig)
-        group128_quant_kernel<kGroupU, true><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        launch(group128_quant_kernel<kGroupU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     else
-        group128_quant_kernel<kGroupU, false><<<grid, kQuantThreads, 0, st>>>(xs, ldx, q, ldq, scales, groups, G);
+        launch(group128_quant_kernel<kGroupU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     return launch_status();
 }
 
@@ -681,8 +663,8 @@ static int run_block128(const void* w, int64_t N, int64_t K, int64_t ldw, uint8_
     const int64_t G = K / 128;
     dim3 grid(unsigned(G), unsigned((N + 127) / 128));
     const uint16_t* ws = static_cast<const uint16_t*>(w);
-    if (e8) block128_quant_kernel<true><<<grid, kQuantThreads, 0, st>>>(ws, N, ldw, qb, ldqb, sb, G);
-    else block128_quant_kernel<false><<<grid, kQuantThreads, 0, st>>>(ws, N, ldw, qb, ldqb, sb, G);
+    if (e8) launch(block128_quant_kernel<true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, ws, N, ldw, qb, ldqb, sb, G);
+    else launch(block128_quant_kernel<false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, ws, N, ldw, qb, ldqb, sb, G);
     return launch_status();
 }
 
@@ -709,7 +691,7 @@ int fp8_act_quant_per_channel(const void* x, int64_t M, int64_t K, int64_t ldx, 
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(M, int64_t(d->sms) * kBlocksPerSm)));
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] per_channel M=%lld K=%lld: grid=%d\n", (long long)M, (long long)K, grid);
-    per_channel_quant_kernel<4><<<grid, kQuantThreads, 0, st>>>(static_cast<const uint16_t*>(x), M, K / 8, ldx,
+    launch(per_channel_quant_kernel<4>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, static_cast<const uint16_t*>(x), M, K / 8, ldx,
                                                             q, ldq, scales);
     return launch_status();
 }
@@ -729,7 +711,7 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
     if (M <= 0 || N <= 0 || K <= 0 || K % 128) return 0;
     DeviceInfo* d = nullptr;
     if (device_info(&d) != FP8Q_OK) return 0;
-    // the ue8m0 and fused GEMMs never run as CTA pairs: size for both plans
+    // the ue8m0 GEMM never runs as CTA pairs: size for both plans
     return std::max(plan_gemm(M, N, K, d->sms).ws_bytes, plan_gemm(M, N, K, d->sms, true).ws_bytes);
 }
 
@@ -742,34 +724,31 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 // mode as in run_gemm.
 static int check_gemm_args(int mode, const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb,
                            int64_t ldb, const float* sb, const void* y, int64_t ldy, int64_t M, int64_t N,
-                           int64_t K, const uint16_t* x, int64_t ldx, bool* empty) {
-    const bool ue8m0 = mode == 2, fused = mode == 4;
+                           int64_t K, bool* empty) {
+    const bool ue8m0 = mode == 2;
     *empty = false;
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
     if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 || N == 0) { *empty = true; return FP8Q_OK; }
-    if ((fused ? !x : (!qa || !sa)) || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
-    if ((fused ? ldx < K : lda < K) || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
-    if ((fused ? (!aligned16(x) || ldx % 8) : (!aligned16(qa) || lda % 16)) ||
-        !aligned16(qb) || !aligned16(y) || ldb % 16 || (ldy * 2) % 16 ||
-        (!ue8m0 && ((!fused && !aligned4(sa)) || !aligned4(sb))))
+    if (!qa || !sa || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+    if (lda < K || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned16(qa) || lda % 16 || !aligned16(qb) || !aligned16(y) || ldb % 16 || (ldy * 2) % 16 ||
+        (!ue8m0 && (!aligned4(sa) || !aligned4(sb))))
         return FP8Q_ERR_MISALIGNED;
     return FP8Q_OK;
 }
 
 static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
                     const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                    void* workspace, size_t workspace_bytes, void* stream, int mode,
-                    const uint16_t* x = nullptr, int64_t ldx = 0, bool pdl = false,
+                    void* workspace, size_t workspace_bytes, void* stream, int mode, bool pdl = false,
                     size_t ws_cap = ~size_t(0)) {
     // mode 0: fp32 block scales; 1: per-tensor fp32 scales; 2: ue8m0 bytes;
-    // 3: per-channel fp32 scales; 4: fp32 block scales with the group-128
-    // quantisation of bf16 tokens x fused in (swapped tiles of <= 32 tokens;
-    // qa and sa unused)
-    const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3, fused = mode == 4;
+    // 3: per-channel fp32 scales.  pdl: the weights do not depend on the
+    // previous kernel on the stream (it writes only qa and sa).
+    const bool per_tensor = mode == 1, ue8m0 = mode == 2, per_channel = mode == 3;
     bool empty = false;
-    int rc = check_gemm_args(mode, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, x, ldx, &empty);
+    int rc = check_gemm_args(mode, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, &empty);
     if (rc != FP8Q_OK || empty) return rc;
     DeviceInfo* d = nullptr;
     rc = device_info(&d);
@@ -780,7 +759,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2 || mode == 4, ws_cap);   // no ue8m0 / fused pairs
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2, ws_cap);   // no ue8m0 pairs
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -790,10 +769,8 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     const uint8_t* Q = pl.swap ? qa : qb;
     const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
     const int64_t ld_p = pl.swap ? ldb : lda, ld_q = pl.swap ? lda : ldb;
-    if (fused && !(pl.swap && pl.bn <= 32)) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (!make_tmap(&tp, P, rows_p, K, ld_p, 128)) return FP8Q_ERR_CUDA;
-    if (fused) tq = tp;                            // the token operand is written by the kernel
-    else if (!make_tmap(&tq, Q, rows_q, K, ld_q, pl.pair ? pl.bn / 2 : pl.bn)) return FP8Q_ERR_CUDA;
+    if (!make_tmap(&tq, Q, rows_q, K, ld_q, pl.pair ? pl.bn / 2 : pl.bn)) return FP8Q_ERR_CUDA;
     GemmParams p;
     p.sa = sa;
     p.sb = sb;
@@ -820,7 +797,6 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     if (staged && (!make_scale_tmap(&tsa, sa, M, p.G, 128) ||
                    !make_scale_tmap(&tsb, sb, (N + 127) / 128, p.G, pl.bn / 128)))
         return FP8Q_ERR_CUDA;
-    if (fused && !make_x_tmap(&tsa, x, M, K, ldx, pl.bn)) return FP8Q_ERR_CUDA;   // the token tiles
     p.wait_budget = wait_budget_cycles();
     p.status_slot = uint8_t(status_slot(d->index, st));
     if (log_enabled())
@@ -829,10 +805,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
                      (long long)M, (long long)N, (long long)K,
                      pl.swap ? "swap" : pl.pair ? "pair" : "normal", staged ? " (staged scales)" : "", pl.bn,
                      pl.stages, pl.splits, pl.units, pl.grid, pl.tail_tiles, pl.tail_splits);
-    if (fused) {
-        if (pl.bn == 16) launch_gemm<16, true, 8, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
-        else launch_gemm<32, true, 7, false, 4>(tp, tq, tsa, tsb, p, pl.grid, st);
-    } else if (per_channel) {
+    if (per_channel) {
         if (pl.pair) {
             if (pl.bn == 256) launch_gemm<256, false, 6, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
             else launch_gemm<128, false, 8, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
@@ -904,12 +877,12 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     if (pl.splits > 1) {
         const int64_t total = M * ((N + 3) / 4);
         const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
-        splitk_reduce_kernel<<<g, 256, 0, st>>>(p.ws, pl.splits, p.M, p.N, pl.ldw, p.y, ldy);
+        launch(splitk_reduce_kernel, dim3(g), dim3(256), 0, st, 1u, p.ws, pl.splits, p.M, p.N, pl.ldw, p.y, ldy);
         rc = launch_status();
     } else if (pl.tail_tiles > 0) {
         const int64_t total = int64_t(pl.tail_tiles) * 128 * (pl.bn / 4);
         const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
-        tail_reduce_kernel<<<g, 256, 0, st>>>(p.ws, pl.tail_tiles, pl.tail_splits, pl.full_tiles,
+        launch(tail_reduce_kernel, dim3(g), dim3(256), 0, st, 1u, p.ws, pl.tail_tiles, pl.tail_splits, pl.full_tiles,
                                               pl.tiles_p, pl.bn, p.M, p.N, p.y, ldy);
         rc = launch_status();
     }
@@ -930,21 +903,13 @@ int fp8_gemm_per_tensor(const uint8_t* qa, int64_t lda, const float* sa, const u
     return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 1);
 }
 
-// ------------------------------------------------------------ fused linear
-// FP8Q_LINEAR selects how fp8_linear_group128 runs (measurement only; every
-// choice computes the same bytes): unset -> quantisation kernel, then the
-// GEMM as a programmatic dependent; "fused" -> quantisation inside the GEMM
-// for swapped tiles of <= 32 tokens; "serial" -> the two kernels without
-// launch overlap.
-static const char* linear_mode() {
-    static const char* v = [] { const char* e = std::getenv("FP8Q_LINEAR"); return e ? e : ""; }();
-    return v;
-}
-static bool linear_in_kernel_quant() { return std::strcmp(linear_mode(), "fused") == 0; }
-static bool linear_without_overlap() { return std::strcmp(linear_mode(), "serial") == 0; }
-
-// Workspace layout when the launch is not fused: codes [M, K], then the
-// group scales [M, K/128] fp32, then the GEMM's split-K partials.
+// ------------------------------------------------------------ one-call linear
+// Group-128 quantisation of x into the workspace, then the block GEMM on
+// it, launched as a programmatic dependent of the quantisation: its
+// producer issues the weight loads of its first pipeline stages (weights
+// do not depend on the quantisation) before it waits for the codes.
+// Workspace layout: codes [M, K], then the group scales [M, K/128] fp32,
+// then the GEMM's split-K partials.
 static size_t round256(size_t b) { return (b + 255) / 256 * 256; }
 
 size_t fp8_linear_group128_workspace_size(int64_t M, int64_t N, int64_t K) {
@@ -952,7 +917,6 @@ size_t fp8_linear_group128_workspace_size(int64_t M, int64_t N, int64_t K) {
     DeviceInfo* d = nullptr;
     if (device_info(&d) != FP8Q_OK) return 0;
     const GemmPlan pl = plan_gemm(M, N, K, d->sms);
-    if (linear_in_kernel_quant() && pl.swap && pl.bn <= 32) return pl.ws_bytes;
     return round256(size_t(M) * size_t(K)) + round256(size_t(M) * size_t(K / 128) * 4) + pl.ws_bytes;
 }
 
@@ -960,19 +924,17 @@ int fp8_linear_group128(const void* x, int64_t ldx, const uint8_t* qb, int64_t l
                         void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream) {
     if (M < 0 || N < 0 || K < 0) return FP8Q_ERR_INVALID_ARG;
-    if (K % 128) return FP8Q_ERR_UNSUPPORTED_SHAPE;
+    if (K % 128 || M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
     if (M == 0 || N == 0) return FP8Q_OK;
+    if (!x || !qb || !sb || !y) return FP8Q_ERR_INVALID_ARG;
+    if (ldx < K || ldb < K || ldy < N) return FP8Q_ERR_INVALID_ARG;
+    if (!aligned16(x) || (ldx * 2) % 16 || !aligned16(qb) || ldb % 16 || !aligned4(sb) || !aligned16(y) ||
+        (ldy * 2) % 16)
+        return FP8Q_ERR_MISALIGNED;
     DeviceInfo* d = nullptr;
     int rc = device_info(&d);
     if (rc != FP8Q_OK) return rc;
     const GemmPlan pl = plan_gemm(M, N, K, d->sms);
-    if (linear_in_kernel_quant() && pl.swap && pl.bn <= 32) {
-        if (log_enabled())
-            std::fprintf(stderr, "[fp8q] linear M=%lld N=%lld K=%lld: group-128 quantisation fused into the GEMM\n",
-                         (long long)M, (long long)N, (long long)K);
-        return run_gemm(nullptr, 0, nullptr, qb, ldb, sb, y, ldy, M, N, K, workspace, workspace_bytes, stream, 4,
-                        static_cast<const uint16_t*>(x), ldx);
-    }
     const size_t need = fp8_linear_group128_workspace_size(M, N, K);
     if (!workspace || workspace_bytes < need) return FP8Q_ERR_WORKSPACE;
     if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -980,9 +942,7 @@ int fp8_linear_group128(const void* x, int64_t ldx, const uint8_t* qb, int64_t l
     float* sa = reinterpret_cast<float*>(qa + round256(size_t(M) * size_t(K)));
     uint8_t* gws = reinterpret_cast<uint8_t*>(sa) + round256(size_t(M) * size_t(K / 128) * 4);
     if ((rc = run_group128(x, M, K, ldx, qa, K, sa, false, stream)) != FP8Q_OK) return rc;
-    // the GEMM starts its weight loads while the quantisation runs
-    return run_gemm(qa, K, sa, qb, ldb, sb, y, ldy, M, N, K, gws, pl.ws_bytes, stream, 0,
-                    nullptr, 0, !linear_without_overlap());
+    return run_gemm(qa, K, sa, qb, ldb, sb, y, ldy, M, N, K, gws, pl.ws_bytes, stream, 0, true);
 }
 
 int fp8_gemm_per_channel(const uint8_t* qa, int64_t lda, const float* sa, const uint8_t* qb, int64_t ldb,
@@ -1005,7 +965,7 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, cons
     // Argument errors first, with fp8_block_gemm's checks and codes, before
     // the device is queried or the launch is planned against the scratch.
     bool empty = false;
-    int rc = check_gemm_args(0, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, nullptr, 0, &empty);
+    int rc = check_gemm_args(0, qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, &empty);
     if (rc != FP8Q_OK || empty) return rc;
     DeviceInfo* d = nullptr;
     rc = device_info(&d);
@@ -1018,7 +978,7 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa, cons
     rc = noalloc_scratch(&scratch);
     if (rc != FP8Q_OK) return rc;
     return run_gemm(qa, lda, sa, qb, ldb, sb, y, ldy, M, N, K, scratch, kNoAllocScratchBytes, stream, 0,
-                    nullptr, 0, false, kNoAllocScratchBytes);
+                    false, kNoAllocScratchBytes);
 }
 
 // ------------------------------------------------------------ status

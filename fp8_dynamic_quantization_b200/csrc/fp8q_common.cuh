@@ -180,6 +180,18 @@ __device__ __forceinline__ void st_stream8(void* p, const uint2& v) {
     asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};" :: "l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
+// Programmatic dependent launch.  The library launches its kernels as
+// programmatic dependents of the work before them on the stream: a kernel
+// first lets its successor begin launching (its CTAs are placed as this
+// kernel's CTAs retire), then waits until its predecessor has completed and
+// that grid's writes are visible, before it touches global memory.  So the
+// launch of each kernel overlaps the tail of the one before it, and stream
+// order is kept.  Launched without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t warp_max(uint32_t v) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));

@@ -16,9 +16,9 @@
 // Warp roles (one CTA per SM, persistent over work units):
 //   warpgroup 0   warp 0: TMA producer (P and Q tiles of one K block per
 //                 pipeline stage); warp 1: TMEM allocation and the single
-//                 thread that issues tcgen05.mma; warps 2-3: the ue8m0
-//                 scale-slot writer (warp 2, scale mode 2) or the token
-//                 quantisers (scale mode 4), otherwise idle.  With several
+//                 thread that issues tcgen05.mma; warp 2: the ue8m0
+//                 scale-slot writer (scale mode 2), otherwise idle; warp 3
+//                 idle.  With several
 //                 promotion warpgroups warpgroup 0 hands registers to them
 //                 (setmaxnreg 48/224 or 56/216 for two, 32/160 for three).
 //   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row)
@@ -48,9 +48,12 @@
 // wave is short and fills the SMs; those partials go to the workspace
 // (tile-local [unit][128][BN] fp32) and tail_reduce_kernel adds them in
 // fixed order into Y.
-// Programmatic dependent launch (p.pdl): the producer issues the weight
-// halves of its first STAGES stages, then waits for the grid that writes A
-// and sa (griddepcontrol.wait); the promotion waits before reading scales.
+// Programmatic dependent launch: every GEMM is launched as a programmatic
+// dependent of the previous kernel on the stream; its prologue (barriers,
+// TMEM allocation, tensor-map prefetch) overlaps that kernel's tail, and
+// every thread waits for it (griddepcontrol.wait) before touching global
+// memory.  With p.pdl set (the previous kernel writes only A and sa), the
+// producer first issues the weight halves of its first STAGES stages.
 
 // Scale mode SM:
 //   0  fp32 block scales, promoted per K block as above.
@@ -71,14 +74,6 @@
 //   3  per-channel scales (sa [M] per row of A, sb [N] per row of B): one
 //      TMEM accumulation per unit; the epilogue multiplies row m by its
 //      scale and column n by the one staged for the tile in shared memory.
-//   4  swapped mode with the group-128 quantisation of the tokens fused in:
-//      A arrives as bf16 (read through the token tensor map, the tmSA
-//      argument).  The producer also copies each K block's bf16
-//      token tile (BN rows x 256 bytes) into a per-stage ring; warps 2-3
-//      quantise it (per-row amax over the block = the 1x128 group, scale =
-//      amax/448, codes), write the codes into the stage's operand slot in
-//      the 128-byte-swizzled layout TMA would produce, and pass sa*sb per
-//      token through an 8-slot ring to the promotion warps.
 #pragma once
 
 #include <cuda.h>
@@ -104,7 +99,7 @@ struct GemmParams {
     // bytes measurably slowed the kernel (2%).
     uint8_t scale_vec4;  // sa/sb rows readable as float4 (G % 4 == 0, 16-byte aligned)
     uint8_t sf_words;    // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
-    uint8_t pdl;         // launched as a programmatic dependent of the kernel producing A and sa
+    uint8_t pdl;         // the weights do not depend on the previous kernel (it produces A and sa)
     uint8_t status_slot; // error word of the launching stream (g_stream_status index)
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
@@ -115,9 +110,6 @@ struct GemmCfg {
     static constexpr bool PT = SM == 1;                        // per-tensor scales
     static constexpr bool MX = SM == 2;                        // ue8m0 scales applied by the MMA
     static constexpr bool PC = SM == 3;                        // per-channel scales
-    static constexpr bool FQ = SM == 4;                        // token quantisation fused in (swapped)
-    static constexpr int kFqSlots = FQ ? 8 : 0;               // ring of per-K-block column scales
-    static constexpr int kXBytes = FQ ? BN * 256 : 0;          // bf16 token tile per stage (FQ)
     // BN is the MMA's N.  PAIR: a CTA pair computes a 256 x BN tile with
     // cta_group::2 MMAs; each CTA holds 128 rows of A and BN/2 rows of B,
     // and its TMEM receives its 128 rows x BN columns of every product.
@@ -148,7 +140,7 @@ struct GemmCfg {
                                    : kNumBuf * BN <= 128 ? 128 : kNumBuf * BN <= 256 ? 256 : 512;
     static constexpr int kMaxUnitKb = 64;                      // K blocks per unit (swapped mode)
     // swapped-mode scale slab (block scales); per-channel: the tile's column scales
-    static constexpr int kSlabFloats = (SWAP && SM == 0) ? BN * kMaxUnitKb : PC ? BN : FQ ? BN * kFqSlots : 0;
+    static constexpr int kSlabFloats = (SWAP && SM == 0) ? BN * kMaxUnitKb : PC ? BN : 0;
     // SS: block scales staged through shared memory.  The producer copies,
     // per group of 4 K blocks, the tile's 128 x 4 row scales and its
     // BN/128 x 4 column-block scales into a ring of kScaleSlots slots.
@@ -158,7 +150,7 @@ struct GemmCfg {
     static constexpr uint32_t kScaleTx = 2048 + 16 * kSbRows;  // bytes one slot receives
     static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
                                          + size_t(kSlabFloats) * 4 + size_t(kScaleSlots) * kScaleSlotBytes
-                                         + size_t(kSfSlots) * kSfSlotBytes + size_t(STAGES) * kXBytes + 512;
+                                         + size_t(kSfSlots) * kSfSlotBytes + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
     static_assert(kCW % 16 == 0, "columns per thread");
     static_assert(!SWAP || BN <= 128, "swapped tiles hold at most 128 tokens");
@@ -168,9 +160,7 @@ struct GemmCfg {
     static_assert(!PAIR || (!SWAP && (BN == 256 || BN == 128)), "CTA pairs compute 256 x 256 or 256 x 128 tiles");
     static_assert(kStageBytes % 1024 == 0, "stage alignment");
     static_assert(kSmemBytes <= 232448, "shared memory");
-    static_assert((2 * STAGES + 2 * kNumBuf + 2 * kScaleSlots + 2 * kSfSlots + 2 * kFqSlots + (FQ ? STAGES : 0)) * 8
-                      + 8 <= 512, "barrier area");
-    static_assert(!FQ || (SWAP && !PAIR && BN <= 32 && BN % 2 == 0), "fused quantisation: swapped tiles of <= 32 tokens");
+    static_assert((2 * STAGES + 2 * kNumBuf + 2 * kScaleSlots + 2 * kSfSlots) * 8 + 8 <= 512, "barrier area");
     static_assert(!SS || (!SWAP && !PAIR && SM == 0 && (BN == 128 || BN == 256)), "staged scales: normal 128/256 tiles");
     static_assert(!MX || (!PAIR && kNumBuf >= 1), "ue8m0 tiles: one CTA, at least one TMEM buffer");
 };
@@ -314,12 +304,11 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmSB,    // column-block scales [NB, G] fp32 (SS only)
                   const GemmParams p) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
-    constexpr bool PT = C::PT, MX = C::MX, PC = C::PC, FQ = C::FQ;
+    constexpr bool PT = C::PT, MX = C::MX, PC = C::PC;
     constexpr bool ONE = PT || MX || PC;  // one TMEM accumulation per unit, no per-K-block promotion
     constexpr int NB = C::kNumBuf;
     constexpr uint32_t kSlots = C::kScaleSlots > 0 ? C::kScaleSlots : 1;   // divisor for the (SS) slot ring
     constexpr uint32_t kSfN = C::kSfSlots > 0 ? C::kSfSlots : 1;         // divisor for the (MX) slot ring
-    constexpr uint32_t kFqN = C::kFqSlots > 0 ? C::kFqSlots : 1;         // divisor for the (FQ) scale ring
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -327,8 +316,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     float* slab = reinterpret_cast<float*>(smem + size_t(STAGES) * C::kStageBytes);
     uint8_t* sring = smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4;   // SS slots
     uint8_t* sfring = sring + size_t(C::kScaleSlots) * C::kScaleSlotBytes;   // MX scale-factor slots
-    uint8_t* xring = sfring + size_t(C::kSfSlots) * C::kSfSlotBytes;          // FQ bf16 token tiles
-    uint64_t* bars = reinterpret_cast<uint64_t*>(xring + size_t(STAGES) * C::kXBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sfring + size_t(C::kSfSlots) * C::kSfSlotBytes);
     uint64_t* full = bars;                        // [STAGES] TMA landed
     uint64_t* empty = bars + STAGES;              // [STAGES] MMA done reading
     uint64_t* tfull = bars + 2 * STAGES;          // [NB] block partial ready in TMEM
@@ -337,12 +325,10 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     uint64_t* sempty = sfull + C::kScaleSlots;     // [kScaleSlots] scale slot read by every promotion warp
     uint64_t* sffull = sempty + C::kScaleSlots;   // [kSfSlots] scale-factor slot written (MX)
     uint64_t* sfempty = sffull + C::kSfSlots;     // [kSfSlots] slot consumed by the MMAs (MX)
-    uint64_t* qfull = sfempty + C::kSfSlots;      // [kFqSlots] token scales written (FQ)
-    uint64_t* qempty = qfull + C::kFqSlots;       // [kFqSlots] token scales read by every promotion warp
-    uint64_t* xfull = qempty + C::kFqSlots;       // [STAGES] token tile landed (FQ)
-    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(xfull + (FQ ? STAGES : 0));
+    uint32_t* tmem_base_smem = reinterpret_cast<uint32_t*>(sfempty + C::kSfSlots);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_smem + 1);
 
+    ptx::griddep_launch_dependents();    // the next kernel on the stream may begin launching
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // CTA pair: rank 0 (the leader) issues the MMAs; both load, both promote.
     const uint32_t rank = PAIR ? ptx::cluster_ctarank() : 0u;
@@ -351,14 +337,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     const int unit_step = PAIR ? int(ptx::num_clusters_x()) : int(gridDim.x);
 
     if (threadIdx.x == 0) {
-        // FQ: a stage is full once the weight copy landed and a quantiser warp wrote the tokens
-        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&full[s], FQ ? 2 : 1); ptx::mbar_init(&empty[s], 1); }
-        for (int i = 0; i < C::kFqSlots; ++i) {
-            ptx::mbar_init(&qfull[i], 1);
-            ptx::mbar_init(&qempty[i], 4 * C::kEpiWG);
-        }
-        if (FQ)
-            for (int i = 0; i < STAGES; ++i) ptx::mbar_init(&xfull[i], 1);
+        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&full[s], 1); ptx::mbar_init(&empty[s], 1); }
         for (int b = 0; b < NB; ++b) {
             ptx::mbar_init(&tfull[b], 1);
             ptx::mbar_init(&tempty[b], (PAIR ? 2 : 1) * 4 * C::kEpiWG);
@@ -388,77 +367,14 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     else __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem_base = *tmem_base_smem;
+    // Nothing above touched global memory.  Wait for the previous kernel on
+    // the stream (programmatic dependent launch) before anything does; only
+    // the producer of a launch whose weights do not depend on that kernel
+    // (p.pdl) issues the weight loads of its first stages before it waits.
+    const bool early_weights = !PAIR && SM == 0 && p.pdl && warp == 0 && lane == 0;
+    if (!early_weights) ptx::griddep_wait();
 
     auto fail = [&]() { *abort_flag = 1; record_error(p.status_slot, 6 /* FP8Q_ERR_TIMEOUT */); };
-
-    // ------------------------------------------ token quantiser (fused mode)
-    // Run by warps 2 and 3; `mine` is this warp's index among them.
-    constexpr uint32_t kQuantWarps = 2;
-    // The warps take K blocks round robin, so kQuantWarps blocks are in
-    // flight.  Within a block, half-warp h owns rows h, h+2, ...: lane c of
-    // the half holds 8 values (chunk c of the 128-wide K block, read from the
-    // bf16 tile in shared memory); 4 shuffles give a row's amax over the
-    // block, i.e. its 1x128 group.  The unit's weight-block scales sit in two
-    // registers per lane (a unit spans <= 64 K blocks) and are fetched by
-    // shuffle.
-    auto quantise = [&](uint32_t mine) {
-        const int c = lane & 15;
-        const int r0 = lane >> 4;
-        uint32_t it = 0, qg = 0;
-        bool stop = false;
-        for (int u = unit0; u < p.units && !stop; u += unit_step) {
-            int tp, tq, kb0, kb1;
-            unit_coords(p, u, tp, tq, kb0, kb1);
-            const float* sbr = p.sb + int64_t(tp) * p.G;
-            const float sb_lo = kb0 + lane < kb1 ? __ldg(sbr + kb0 + lane) : 0.0f;
-            const float sb_hi = kb0 + 32 + lane < kb1 ? __ldg(sbr + kb0 + 32 + lane) : 0.0f;
-            for (int kb = kb0; kb < kb1; ++kb, ++it, ++qg) {
-                if (it % kQuantWarps != mine) continue;               // another warp's block
-                const int s = it % STAGES;
-                const uint32_t ph = (it / STAGES) & 1;
-                const uint32_t slot = qg % kFqN, sph = (qg / kFqN) & 1;
-                const int kbl = kb - kb0;
-                const float sbv = __shfl_sync(0xFFFFFFFFu, kbl < 32 ? sb_lo : sb_hi, kbl & 31);
-                bool ok = true;
-                // the tile landing implies the stage's operand slot is free
-                // (its copy was issued after the stage emptied)
-                if (lane == 0)
-                    ok = ptx::mbar_wait(&xfull[s], ph, p.wait_budget) &&
-                         ptx::mbar_wait(&qempty[slot], sph ^ 1, p.wait_budget);
-                ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-                if (!ok) { if (lane == 0) fail(); stop = true; break; }
-                __syncwarp();
-                const uint8_t* xs = xring + size_t(s) * C::kXBytes;              // BN rows x 256 B
-                uint8_t* qdst = tiles + size_t(s) * C::kStageBytes + C::kPBytes;   // BN rows x 128 B
-                // rows r0, r0+2, ...: independent chains, interleaved by full unrolling
-                constexpr int kRows = BN / 2;
-                uint4 v[kRows];
-                uint32_t a[kRows];
-#pragma unroll
-                for (int i = 0; i < kRows; ++i) {
-                    v[i] = *reinterpret_cast<const uint4*>(xs + (r0 + 2 * i) * 256 + c * 16);
-                    a[i] = absmax8(v[i]);
-                }
-#pragma unroll
-                for (int o = 8; o >= 1; o >>= 1)
-#pragma unroll
-                    for (int i = 0; i < kRows; ++i) a[i] = max(a[i], __shfl_xor_sync(0xFFFFFFFFu, a[i], o));
-#pragma unroll
-                for (int i = 0; i < kRows; ++i) {
-                    const int r = r0 + 2 * i;
-                    const float sc = scale_from_amax_bits(a[i]);
-                    // 128-byte swizzle: 16-byte chunk j of row r sits at chunk j ^ (r % 8)
-                    *reinterpret_cast<uint2*>(qdst + r * 128 + ((((c >> 1) ^ (r & 7)) << 4) | ((c & 1) << 3))) =
-                        quant8(v[i], make_scale(sc));
-                    if (c == 0) slab[slot * BN + r] = sc * sbv;
-                }
-                ptx::fence_proxy_async_shared();
-                __syncwarp();
-                if (lane == 0) { ptx::mbar_arrive(&full[s]); ptx::mbar_arrive(&qfull[slot]); }
-            }
-        }
-        __syncwarp();
-    };
 
     if (warp < 4) {
         if (C::kEpiWG > 1) ptx::regs_dec<C::kRegWG0>();
@@ -488,8 +404,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 }
             }
             __syncwarp();
-        } else if (FQ && (warp == 2 || warp == 3)) {
-            quantise(uint32_t(warp - 2));
         } else if (warp == 0 && lane == 0) {
             // -------------------------------------------------------- producer
             // PDL: the weights do not depend on the previous kernel, so the
@@ -544,11 +458,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                         if (leader) ptx::mbar_arrive_expect_tx(&full[s], 2 * C::kStageBytes);
                         ptx::tma_load_2d_pair(dst, &tmP, bar0, kb * 128, prow);
                         ptx::tma_load_2d_pair(dst + C::kPBytes, &tmQ, bar0, kb * 128, qrow);
-                    } else if (FQ) {                  // codes come from warps 2-3, from the bf16 tile
-                        ptx::mbar_arrive_expect_tx(&full[s], C::kPBytes);
-                        ptx::tma_load_2d(dst, &tmP, &full[s], kb * 128, prow);
-                        ptx::mbar_arrive_expect_tx(&xfull[s], C::kXBytes);
-                        ptx::tma_load_2d(xring + size_t(s) * C::kXBytes, &tmSA, &xfull[s], kb * 128, qrow);
                     } else {
                         ptx::mbar_arrive_expect_tx(&full[s], C::kStageBytes);
                         ptx::tma_load_2d(dst, &tmP, &full[s], kb * 128, prow);
@@ -561,9 +470,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 const uint32_t first = it > STAGES ? it - STAGES : 0;
                 for (uint32_t j = first; j < it; ++j)
                     ptx::mbar_wait(&full[j % STAGES], (j / STAGES) & 1, 100000000LL);
-                if (FQ)
-                    for (uint32_t j = first; j < it; ++j)
-                        ptx::mbar_wait(&xfull[j % STAGES], (j / STAGES) & 1, 100000000LL);
                 const uint32_t sfirst = sg > uint32_t(C::kScaleSlots) ? sg - C::kScaleSlots : 0;
                 for (uint32_t g = sfirst; g < sg; ++g)
                     ptx::mbar_wait(&sfull[g % kSlots], (g / kSlots) & 1, 100000000LL);
@@ -658,7 +564,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     } else {
         // ------------------------------------------------------------ promotion
         if (C::kEpiWG > 1) ptx::regs_inc<C::kRegEpi>();
-        if (p.pdl) ptx::griddep_wait();           // the scales come from the previous kernel
         const int e = warp - 4;                   // 0 .. 4*kEpiWG-1
         const int quarter = warp & 3;             // TMEM lane quarter this warp may access
         const int chalf = e >> 2;                 // which kCW-column slice
@@ -668,7 +573,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         const bool vec4 = p.scale_vec4 != 0;
         uint32_t c = 0;
         uint32_t sg = 0;                          // scale groups consumed (SS)
-        uint32_t fqg = 0;                         // token-scale slots consumed (FQ)
         uint64_t acc2[C::kCW / 2];
         // the leader's tempty barriers, as cluster addresses (pair mode)
         const uint32_t tempty0 = PAIR ? ptx::mapa_shared(ptx::smem_u32(tempty), 0) : 0u;
@@ -759,12 +663,6 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16)
                                        + buf * BN + chalf * C::kCW;
                 const float* sl = slab + (kb - kb0) * BN + chalf * C::kCW;
-                uint32_t fq_slot = 0;
-                if (FQ) {
-                    fq_slot = fqg % kFqN;
-                    if (!ptx::mbar_wait(&qfull[fq_slot], (fqg / kFqN) & 1, p.wait_budget)) { fail(); ok = false; break; }
-                    sl = slab + fq_slot * BN + chalf * C::kCW;
-                }
                 // Loads of this thread's kCW columns in chunks of at most 64;
                 // the TMEM buffer is released as soon as the last chunk has
                 // landed, then that chunk's FMAs run.
@@ -785,13 +683,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                             else ptx::mbar_arrive(&tempty[buf]);
                         }
                     }
-                    if (SWAP && (SM == 0 || FQ)) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
+                    if (SWAP && SM == 0) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
                     else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
-                }
-                if (FQ) {                                 // this K block's token scales are read
-                    __syncwarp();
-                    if (lane == 0) ptx::mbar_arrive(&qempty[fq_slot]);
-                    ++fqg;
                 }
             }
             if (!ok) break;
@@ -962,6 +855,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 __global__ void __launch_bounds__(256)
 splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int64_t ldw,
                      uint16_t* __restrict__ y, int64_t ldy) {
+    pdl_begin();
     const int64_t cols4 = (N + 3) / 4;
     const int64_t total = int64_t(M) * cols4;
     for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < total;
@@ -995,6 +889,7 @@ splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int
 __global__ void __launch_bounds__(256)
 tail_reduce_kernel(const float* __restrict__ ws, int tail_tiles, int splits, int full_tiles, int tiles_p,
                    int bn, int M, int N, uint16_t* __restrict__ y, int64_t ldy) {
+    pdl_begin();
     const int quads = bn / 4;
     const int64_t per_tile = int64_t(128) * quads;
     const int64_t total = int64_t(tail_tiles) * per_tile;

@@ -56,8 +56,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
                       uint8_t* __restrict__ q, int64_t ldq,
                       void* __restrict__ scales, int64_t groups, int64_t G) {
-    // a GEMM launched as a programmatic dependent may start its weight loads now
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    pdl_begin();   // a GEMM launched after this one may start its weight loads now
     const int sub = threadIdx.x & 7;
     const int64_t g_first = (int64_t(blockIdx.x) * kQuantThreads + threadIdx.x) >> 3;
     const int64_t g_stride = (int64_t(gridDim.x) * kQuantThreads) >> 3;
@@ -115,6 +114,7 @@ template <int U, bool CONTIG>
 __global__ void __launch_bounds__(kQuantThreads)
 amax_partial_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
                     int64_t ldx, uint32_t* __restrict__ partials) {
+    pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
     uint32_t m = 0;
@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, int64_t ldx,
              const uint32_t* __restrict__ partials, int nparts,
              uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scale_out) {
+    pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     uint32_t m = 0;
     for (int i = threadIdx.x; i < nparts; i += kQuantThreads)
@@ -208,6 +209,7 @@ __global__ void __launch_bounds__(NT)
 per_tensor_cluster_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
                           int64_t ldx, uint8_t* __restrict__ q, int64_t ldq,
                           float* __restrict__ scale_out) {
+    pdl_begin();
     constexpr int kClusterThreads = NT;
     __shared__ uint32_t red[kClusterThreads / 32];
     __shared__ uint32_t part;                     // this CTA's partial max
@@ -255,6 +257,7 @@ per_tensor_cluster_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t 
 // out = max(partials[0:n]); one CTA.
 __global__ void __launch_bounds__(kQuantThreads)
 reduce_partials_kernel(const uint32_t* __restrict__ partials, int n, uint32_t* __restrict__ out) {
+    pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     uint32_t m = 0;
     for (int i = threadIdx.x; i < n; i += kQuantThreads) m = max(m, __ldcg(partials + i));
@@ -264,6 +267,7 @@ reduce_partials_kernel(const uint32_t* __restrict__ partials, int n, uint32_t* _
 
 // scale = amax / 448 from an amax word, for an empty apply.
 __global__ void scale_only_kernel(const uint32_t* __restrict__ amax_bits, float* __restrict__ scale) {
+    pdl_begin();
     if (threadIdx.x == 0) *scale = scale_from_amax_bits(*amax_bits & 0x7FFFu);
 }
 
@@ -279,6 +283,7 @@ template <int U>
 __global__ void __launch_bounds__(kQuantThreads)
 per_channel_quant_kernel(const uint16_t* __restrict__ x, int64_t M, int64_t vpr, int64_t ldx,
                          uint8_t* __restrict__ q, int64_t ldq, float* __restrict__ scales) {
+    pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     if (vpr <= int64_t(U) * kQuantThreads) {
         uint4 cur[U], nxt[U];
@@ -340,6 +345,7 @@ template <bool E8 = false>   // E8: E8M0 scale bytes in `sb` (ue8m0 variant)
 __global__ void __launch_bounds__(kQuantThreads)
 block128_quant_kernel(const uint16_t* __restrict__ w, int64_t N, int64_t ldw,
                       uint8_t* __restrict__ q, int64_t ldq, void* __restrict__ sb, int64_t G) {
+    pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t kb = blockIdx.x, nb = blockIdx.y;
     uint4 v[8];

@@ -49,10 +49,16 @@
  *     (NaN codes, or signed zeros for finite x over an infinite scale).
  *   - Determinism: the same inputs give the same bytes, whatever the
  *     launch configuration chosen.
+ *   - Launches: every kernel is launched as a programmatic dependent of the
+ *     work before it on `stream`.  It may be placed on the GPU while the
+ *     previous kernel finishes, and waits for that kernel to complete
+ *     before it touches global memory, so stream order holds as usual and
+ *     the gap between back-to-back kernels shrinks.
  *   - Environment: FP8Q_LOG=1 prints the launch chosen for every call to
  *     stderr.  FP8Q_GEMM_TILE forces a GEMM launch mode and
  *     FP8Q_PER_TENSOR_PATH=twopass the two-pass per-tensor path (measurement);
- *     FP8Q_LINEAR=fused|serial how fp8_linear_group128 runs (measurement);
+ *     FP8Q_PDL=0 launches every kernel without programmatic dependent
+ *     launch (measurement; see "Launches" below);
  *     FP8Q_WAIT_BUDGET_CYCLES bounds the GEMM's device-side waits (fault
  *     testing; fp8q_set_wait_budget_cycles changes it at run time); these
  *     are read once per process.  No environment variable changes the
@@ -149,10 +155,10 @@ int fp8_weight_quant_block128(const void* w, int64_t N, int64_t K, int64_t ldw,
                               uint8_t* qb, int64_t ldqb, float* sb, void* stream);
 
 /* ------------------------------------------------------------------ */
-/* The dynamic FP8 linear with the activation quantisation fused into   */
-/* the GEMM ([P1] "Analyzing FP8 Quantization Sensitivity": act_quant   */
-/* produces the scales that feed fp8_gemm, and its latency matters at   */
-/* small batch).                                                         */
+/* The dynamic FP8 linear in one call: activation quantisation, then   */
+/* the GEMM on its codes ([P1] "Analyzing FP8 Quantization Sensitivity": */
+/* act_quant produces the scales that feed fp8_gemm, and its latency     */
+/* matters at small batch).                                              */
 /* ------------------------------------------------------------------ */
 
 /* Workspace bytes fp8_linear_group128 needs for (M, N, K) on the current
@@ -164,17 +170,12 @@ size_t fp8_linear_group128_workspace_size(int64_t M, int64_t N, int64_t K);
  *   x : bf16 [M,K] (row stride ldx, a multiple of 8; 16-byte aligned)
  *   qb: E4M3 [N,K] (row stride ldb), sb: fp32 [ceil(N/128), K/128]
  *   y : bf16 [M,N] (row stride ldy)
- * By default the quantisation kernel runs first and the GEMM is launched as
- * its programmatic dependent: the GEMM starts while the quantisation runs,
+ * The quantisation kernel runs first and the GEMM is launched as its
+ * programmatic dependent: the GEMM starts while the quantisation runs,
  * issues the weight halves of its first pipeline stages, and waits for the
  * quantisation only before reading the codes and scales (kept in the
- * workspace).  With FP8Q_LINEAR=fused, launches that use swapped tiles of
- * at most 32 tokens quantise each 128-wide K block of the tokens inside the
- * GEMM instead, writing the codes straight into shared memory (measured
- * slower on B200: the per-CTA quantisation is repeated by every CTA and
- * cannot keep pace with the weight stream).  FP8Q_LINEAR=serial runs the two
- * kernels without overlap.  Every choice gives the same bytes.  Errors as
- * fp8_block_gemm. */
+ * workspace).  Argument errors as fp8_act_quant_group128 and
+ * fp8_block_gemm; FP8Q_ERR_WORKSPACE for a missing or short workspace. */
 int fp8_linear_group128(const void* x, int64_t ldx, const uint8_t* qb, int64_t ldb,
                         const float* sb, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
                         void* workspace, size_t workspace_bytes, void* stream);
@@ -251,7 +252,10 @@ size_t fp8_block_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
  * call then enqueues two kernels); results are deterministic for a given
  * shape and device.  A bounded device wait that gives up records
  * FP8Q_ERR_TIMEOUT in the error word of `stream`, read by
- * fp8q_get_last_device_status (or fp8q_device_status for every stream). */
+ * fp8q_get_last_device_status (or fp8q_device_status for every stream);
+ * the call's output is then unspecified (the GEMM kernel stops writing it,
+ * but a split-K or split-tail reduce that follows may write sums of
+ * partials that were never computed). */
 int fp8_block_gemm(const uint8_t* qa, int64_t lda, const float* sa,
                    const uint8_t* qb, int64_t ldb, const float* sb,
                    void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,

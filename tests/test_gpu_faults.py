@@ -59,12 +59,13 @@ from fp8_dynamic_quantization_b200 import _abi, inputs
 lib = _abi.load()
 dev = torch.device("cuda:0")
 fq.device_status(reset=True)
-qa, sa, qb, sb = inputs.gemm_operands(256, 1024, 1024, seed=7)
+# whole tiles, no split-K: the GEMM kernel is the only writer of Y
+qa, sa, qb, sb = inputs.gemm_operands(4096, 2048, 1024, seed=7)
 ops = [torch.from_numpy(a).to(dev) for a in (qa, sa, qb, sb)]
 torch.cuda.synchronize()
 sa_, sb_ = torch.cuda.Stream(), torch.cuda.Stream()
-ya = torch.full((256, 1024), 3.0, dtype=torch.bfloat16, device=dev)
-yb = torch.full((256, 1024), 3.0, dtype=torch.bfloat16, device=dev)
+ya = torch.full((4096, 2048), 3.0, dtype=torch.bfloat16, device=dev)
+yb = torch.full((4096, 2048), 3.0, dtype=torch.bfloat16, device=dev)
 lib.fp8q_set_wait_budget_cycles(0)               # stream A's GEMM gives up at its first wait
 with torch.cuda.stream(sa_):
     fq.block_gemm(*ops, out=ya)

@@ -1,10 +1,10 @@
-"""GPU parity of the one-call linear (fp8_linear_group128) in its three
-launch forms -- quantisation then GEMM as a programmatic dependent (the
-default), quantisation inside the GEMM for skinny M (FP8Q_LINEAR=fused), and
-the two kernels without overlap (FP8Q_LINEAR=serial): each is bit-identical
-to act_quant_group128 followed by block_gemm, and within the GEMM tolerance
-of the oracle's quantisation followed by its block GEMM.  FP8Q_LINEAR is read
-once per process, so each form runs in a child process."""
+"""GPU parity of the one-call linear (fp8_linear_group128): group-128
+quantisation, then the block GEMM launched as its programmatic dependent
+(weight loads start before the codes are ready), and the same call with
+programmatic dependent launch switched off (FP8Q_PDL=0, read once per
+process, hence child processes).  Each is bit-identical to
+act_quant_group128 followed by block_gemm, and within the GEMM tolerance of
+the oracle's quantisation followed by its block GEMM."""
 import os
 import subprocess
 import sys
@@ -62,8 +62,8 @@ print("ok")
 '''
 
 
-@pytest.mark.parametrize("form", ["", "fused", "serial"])
-def test_linear_forms(gpu, cuda_lib, oracle_mod, form):
-    env = dict(os.environ, FP8Q_LINEAR=form)
+@pytest.mark.parametrize("pdl", ["1", "0"])
+def test_linear_forms(gpu, cuda_lib, oracle_mod, pdl):
+    env = dict(os.environ, FP8Q_PDL=pdl)
     r = subprocess.run([sys.executable, "-c", CHILD, ROOT], env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
