@@ -11,13 +11,21 @@ Weight quantisation is an offline step and is not timed.  Inputs per step
 (X and the three weights, 419 MB) exceed the 126 MB L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    python bench.py --op gemm --m 4096 --n 7168 --k 7168 [--reps R] [--modes cold,graph]
 
 Prints ONE JSON line (rank 0).  `value` is the whole-job GEMM throughput of
 the step (2*M*sum(N)*K flops over the device-timed step, all ranks);
-per-kernel times, GB/s and TFLOP/s are in `kernels`.  `--impl reference`
-times the CPU oracle on the host cores on a bounded sample of the same
-workload.  Multi-GPU (torchrun): every rank runs its own batch (weak scaling,
-no collective on the data path); time = max over ranks.
+per-kernel times inside the step are in `kernels`, and `workloads` holds
+every other workload's kernels timed on their own (CUDA-graph replay, as the
+pages timed their amax kernel, and with L2 flushed for the large ones).
+`--impl reference` times the CPU oracle on the host cores on a bounded
+sample of the same workload.  Multi-GPU (torchrun): every rank runs its own
+batch (weak scaling, no collective on the data path); time = max over ranks.
+With more than one rank the row-sharded per-tensor quantisation (local amax,
+one 4-byte MAX all-reduce, local apply) is also timed.
+
+`--op` times one operation at one shape and prints one JSON line per timing
+mode (the commands behind the ncu summaries in profiles/ use it).
 """
 from __future__ import annotations
 
@@ -44,6 +52,11 @@ WORKLOAD = ("prefill linear step: bf16 X[4096,7168] -> per-tensor quant (amax+ap
             "group-128 quant -> block-scaled FP8 GEMM vs B[N,7168] for N in {7168,18432,24576}")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FP8_OVER_BF16 = 2.0            # nominal dense ratio 4.5 / 2.25 PFLOP/s
+L2_BYTES = 126 * 2 ** 20
+# The pages' B200 per-tensor amax kernel (fixed-size grid replaced by an
+# input-sized one), us per call under CUDA graph, K = 2048 ("Size the
+# per-tensor FP8 dynamic-quant amax grid to the input", Test Coverage).
+PAGE_AMAX_US = {1: 4.1, 64: 4.1, 256: 6.1, 1024: 6.1, 65536: 43.0}
 
 
 def gemm_flops(m=M, ns=NS, k=K):
@@ -51,8 +64,15 @@ def gemm_flops(m=M, ns=NS, k=K):
 
 
 # Algorithmic bytes per launch (what the method must move at least once).
-def bytes_per_tensor(m=M, k=K):       # amax read 2B + apply read 2B + write 1B per element
-    return 5.0 * m * k + 4
+def bytes_per_tensor(m=M, k=K, unique=False):
+    """amax read 2 B + apply read 2 B + code write 1 B per element; with
+    unique=True the second read is not counted (3 B/element: the tensor
+    fits in L2, so the apply pass can re-read it from there)."""
+    return (3.0 if unique else 5.0) * m * k + 4
+
+
+def bytes_amax(m, k):
+    return 2.0 * m * k
 
 
 def bytes_group128(m=M, k=K):         # read 2B + write 1B per element + one fp32 per 128
@@ -145,14 +165,15 @@ def parse_clock_rows(text, t0=None, t1=None):
 
 
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 50 ms; the summary
-    keeps the samples stamped inside the timed region."""
+    """nvidia-smi clocks / throttle reasons sampled every `interval_ms`; the
+    summary keeps the samples stamped inside the timed region."""
     QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, index: int):
+    def __init__(self, index, interval_ms: int = 10):
         self.index = index
+        self.interval_ms = interval_ms
         self.proc = None
         self.t0 = self.t1 = None
 
@@ -160,11 +181,11 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "50"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.interval_ms)],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
-        time.sleep(0.1)                      # first samples before the timed region
+        time.sleep(0.3)                      # first samples before the timed region
 
     def mark(self, begin: bool):
         """Host wall-clock bounds of the timed region."""
@@ -191,6 +212,217 @@ def host_cores():
         return len(os.sched_getaffinity(0))
     except AttributeError:
         return os.cpu_count()
+
+
+# ---------------------------------------------------------------- timers
+class Timer:
+    """Device time of one call, CUDA events on the launching stream.
+
+    cold : an L2 flush (reading a 256 MB buffer, which leaves only clean
+           lines in L2) and a GPU sleep before every call, outside the timed
+           interval (the sleep hides the host's launch overhead); median of
+           `reps` calls.
+    graph: `reps` calls captured in one CUDA graph and replayed; time / reps
+           (how the pages timed their amax kernel; inputs that fit in L2 stay
+           L2-warm)."""
+
+    def __init__(self, dev):
+        self.dev = dev
+        self.flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def cold(self, fn, reps):
+        fn()                          # untimed: first-call set-up (workspace, tensor maps)
+        torch.cuda.synchronize()
+        ts = []
+        for _ in range(reps):
+            self.flush_buf.max()
+            torch.cuda._sleep(200_000)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3)
+        return statistics.median(ts)
+
+    def graph(self, fn, reps):
+        fn()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            fn()                      # populate per-stream workspace caches
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        b.synchronize()
+        del g
+        return a.elapsed_time(b) * 1e3 / reps
+
+
+# ---------------------------------------------------------------- operations
+def _dev_codes(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev).view(torch.float8_e4m3fn)
+
+
+def _dev(a, dev):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+
+
+def _out(m, n, dev):
+    """bf16 [m, n] output with a 16-byte row pitch."""
+    return torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
+
+
+def make_op(op, m, n, k, dev):
+    """(callable, algorithmic bytes, flops or None, extra record fields) for
+    one operation at one shape, on seeded synthetic inputs of its workload."""
+    import fp8_dynamic_quantization_b200 as fq
+    if op == "per_tensor":
+        x = inputs.activations_per_tensor(m, k=k).to(dev)
+        return (lambda: fq.act_quant_per_tensor(x)), bytes_per_tensor(m, k), None, {
+            "GB/s_basis": "5 B/element (amax read + apply read + code write)",
+            "unique_bytes": bytes_per_tensor(m, k, unique=True)}
+    if op == "amax":
+        x = inputs.activations_per_tensor(m, k=k).to(dev)
+        return (lambda: fq.act_amax(x)), bytes_amax(m, k), None, {}
+    if op == "group128":
+        x = inputs.activations_group(m, k=k).to(dev)
+        return (lambda: fq.act_quant_group128(x)), bytes_group128(m, k), None, {}
+    if op == "group128_ue8m0":
+        x = inputs.activations_group(m, k=k).to(dev)
+        return (lambda: fq.act_quant_group128_ue8m0(x)), 3.0 * m * k + m * (k // 128), None, {}
+    if op == "per_channel":
+        x = inputs.activations_per_tensor(m, k=k).to(dev)
+        return (lambda: fq.act_quant_per_channel(x)), 3.0 * m * k + 4.0 * m, None, {}
+    flops = 2.0 * m * n * k
+    if op == "gemm":
+        qa, sa, qb, sb = inputs.gemm_operands(m, n, k)
+        tqa, tqb, tsa, tsb = _dev_codes(qa, dev), _dev_codes(qb, dev), _dev(sa, dev), _dev(sb, dev)
+        y = _out(m, n, dev)
+        return (lambda: fq.block_gemm(tqa, tsa, tqb, tsb, out=y)), bytes_gemm(m, n, k), flops, {}
+    if op in ("gemm_pt", "gemm_pc", "gemm_ue8m0"):
+        qa, _, qb, _ = inputs.gemm_operands(m, n, k)
+        tqa, tqb = _dev_codes(qa, dev), _dev_codes(qb, dev)
+        y = _out(m, n, dev)
+        g = inputs.rng(m + n)
+        if op == "gemm_pt":
+            sa, sb = torch.tensor([0.01], device=dev), torch.tensor([0.02], device=dev)
+            return (lambda: fq.gemm_per_tensor(tqa, sa, tqb, sb, out=y)), \
+                m * k + n * k + 8.0 + 2.0 * m * n, flops, {}
+        if op == "gemm_pc":
+            sa = _dev(g.uniform(1e-3, 1e-1, m).astype(np.float32), dev)
+            sb = _dev(g.uniform(1e-3, 1e-1, n).astype(np.float32), dev)
+            return (lambda: fq.gemm_per_channel(tqa, sa, tqb, sb, out=y)), \
+                m * k + n * k + 4.0 * (m + n) + 2.0 * m * n, flops, {}
+        sa = _dev(g.integers(115, 135, (m, k // 128)).astype(np.uint8), dev)
+        sb = _dev(g.integers(115, 135, ((n + 127) // 128, k // 128)).astype(np.uint8), dev)
+        return (lambda: fq.block_gemm_ue8m0(tqa, sa, tqb, sb, out=y)), \
+            m * k + n * k + m * k / 128 + ((n + 127) // 128) * k / 128 + 2.0 * m * n, flops, {}
+    if op == "linear":
+        # the one-call group-128 linear: quantisation kernel, then the GEMM
+        # launched as its programmatic dependent
+        x = inputs.activations_group(m, k=k).to(dev)
+        qb, sb = inputs.weight_operands(n, k)
+        tqb, tsb = _dev_codes(qb, dev), _dev(sb, dev)
+        y = _out(m, n, dev)
+        return (lambda: fq.linear_fused(x, tqb, tsb, out=y)), \
+            2.0 * m * k + n * k + 4.0 * ((n + 127) // 128) * (k // 128) + 2.0 * m * n, flops, {}
+    raise ValueError(op)
+
+
+def time_op(timer, op, m, n, k, dev, modes, reps, hbm, fp8_peak):
+    fn, nbytes, flops, extra = make_op(op, m, n, k, dev)
+    out = []
+    for mode in modes:
+        us = getattr(timer, mode)(fn, reps)
+        rec = {"op": op, "M": m, "N": n, "K": k, "mode": mode, "us": us,
+               "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm}
+        if "unique_bytes" in extra:
+            rec["GB/s_unique"] = extra["unique_bytes"] / us / 1e3
+            rec["frac_hbm_unique"] = rec["GB/s_unique"] / hbm
+        if flops:
+            rec["TFLOP/s"] = flops / us / 1e6
+            rec["frac_fp8"] = flops / us / 1e6 / fp8_peak
+        out.append(rec)
+    del fn
+    return out
+
+
+def fp8_peak_cublaslt(dev, n=8192):
+    """cuBLASLt's per-tensor-scaled FP8 GEMM (torch._scaled_mm, E4M3 in,
+    bf16 out) at n^3 on random data: best of 10 calls, in TFLOP/s.  The
+    measured denominator for FP8 contractions on this GPU."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    a = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(n, n, device=dev, generator=g).to(torch.float8_e4m3fn)
+    one = torch.tensor(1.0, device=dev)
+
+    def f():
+        return torch._scaled_mm(a, b.t(), scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(5):
+        f()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        f()
+        e1.record()
+        e1.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
+
+
+def workload_table(dev, hbm, fp8_peak, reps=20):
+    """Every workload's kernels timed on their own (graph replay; L2-flushed
+    'cold' timing too where the data exceed L2)."""
+    timer = Timer(dev)
+    rows = []
+
+    def add(op, m, n, k, big):
+        modes = ["graph", "cold"] if big else ["graph"]
+        rows.extend(time_op(timer, op, m, n, k, dev, modes, reps, hbm, fp8_peak))
+    # workload 1: the tiny linear layer
+    add("per_tensor", 64, 0, 2048, False)
+    add("group128", 64, 0, 2048, False)
+    add("gemm", 64, 2048, 2048, False)
+    # workload 2: per-tensor sweep, whole path and the amax alone (the pages' kernel)
+    for m in (1, 64, 256, 1024, 65536):
+        big = m * 2048 * 2 > L2_BYTES // 2
+        add("per_tensor", m, 0, 2048, big)
+        before = len(rows)
+        add("amax", m, 0, 2048, big)
+        for r in rows[before:]:
+            r["page_amax_us"] = PAGE_AMAX_US[m]
+    # workload 3: group-128 sweep
+    for m in (1, 32, 4096, 16384):
+        add("group128", m, 0, 7168, m >= 4096)
+    # workload 4: decode GEMM
+    for m in (1, 16, 64, 256):
+        for n in (2048, 7168, 18432):
+            add("gemm", m, n, 7168, n == 18432)
+    # the other scale formats and the one-call linear, decode and prefill
+    for op in ("gemm_pt", "gemm_ue8m0", "gemm_pc"):
+        add(op, 16, 18432, 7168, False)
+        add(op, 4096, 18432, 7168, False)
+    add("linear", 16, 18432, 7168, False)
+    add("linear", 4096, 18432, 7168, False)
+    for op in ("group128_ue8m0", "per_channel"):
+        add(op, 16384, 0, 7168, True)
+    del timer
+    return rows
 
 
 # ---------------------------------------------------------------- CPU oracle
@@ -255,6 +487,26 @@ def reference_arm(args, rank, world):
 
 
 # ---------------------------------------------------------------- GPU arm
+def sharded_per_tensor(x, dist, steps, warmup, stream):
+    """Row-sharded per-tensor quantisation across the ranks (each rank's X is
+    its shard): local amax, one 4-byte MAX all-reduce over NCCL, local
+    apply.  Device time per call, max over ranks."""
+    import fp8_dynamic_quantization_b200 as fq
+    for _ in range(warmup):
+        fq.per_tensor_sharded(x)
+    torch.cuda.synchronize()
+    dist.barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        fq.per_tensor_sharded(x)
+    b.record(stream)
+    torch.cuda.synchronize()
+    t = torch.tensor([a.elapsed_time(b) / steps], dtype=torch.float64, device=x.device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def our_arm(args, rank, world, local_rank):
     import fp8_dynamic_quantization_b200 as fq
     lib = fq.library()
@@ -310,7 +562,7 @@ def our_arm(args, rank, world, local_rank):
     clocks.mark(True)
     start.record(stream)
     for s in range(args.steps):
-        step(events[s])
+        step()
     end.record(stream)
     torch.cuda.synchronize(dev)
     clocks.mark(False)
@@ -321,6 +573,13 @@ def our_arm(args, rank, world, local_rank):
     ms = start.elapsed_time(end)
     if fq.device_status() != 0:
         raise RuntimeError("device-side error during the timed steps")
+
+    # Per-kernel times: a second pass of the same steps with an event between
+    # every two calls (the timed region above has none, so that each launch
+    # can overlap the tail of the one before it).
+    for s in range(args.steps):
+        step(events[s])
+    torch.cuda.synchronize(dev)
 
     # per-kernel averages (ms) from the in-stream events
     def avg(i, j):
@@ -399,33 +658,71 @@ def our_arm(args, rank, world, local_rank):
         e2e_ms = float(t.item())
     h2d = x.numel() * 2
     d2h = sum(M * n * 2 for n in NS)
+    del x_host, y_host, x_devs, y_devs
 
+    # ------------------------------------------------------------ the one exchange (N > 1)
+    sharded_ms = None
+    if dist is not None:
+        sharded_ms = sharded_per_tensor(x, dist, max(10, args.steps), args.warmup, stream)
+
+    peaks, peak_src = load_peaks()
     result = None
+    table = None
+    fp8_meas = None
+    if rank == 0 and not args.no_kernels and world == 1:
+        del ys
+        torch.cuda.empty_cache()
+        fp8_meas = fp8_peak_cublaslt(dev)
+        table = workload_table(dev, peaks["hbm_gbs"], peaks["bf16_tflops"] * FP8_OVER_BF16)
     if rank == 0:
-        peaks, peak_src = load_peaks()
         step_ms = ms / args.steps
         total_flops = gemm_flops() * world
         value = total_flops / (step_ms * 1e-3) / 1e12
+        hbm = peaks["hbm_gbs"]
+        t_pt = k_ms["per_tensor_quant"]
         kernels = {
-            "per_tensor_quant": {"ms": k_ms["per_tensor_quant"],
-                                 "GB/s": bytes_per_tensor() / (k_ms["per_tensor_quant"] * 1e-3) / 1e9},
+            "timing": "per-kernel: in-stream events between the calls of a second pass over the same "
+                      "steps; sum of these can exceed ms_per_step (the events stop each launch from "
+                      "overlapping the previous kernel's tail)",
+            "per_tensor_quant": {
+                "ms": t_pt,
+                "GB/s": bytes_per_tensor() / (t_pt * 1e-3) / 1e9,
+                "GB/s_unique": bytes_per_tensor(unique=True) / (t_pt * 1e-3) / 1e9,
+                "basis": "GB/s at 5 B/element (amax read, apply read, code write); GB/s_unique at "
+                         "3 B/element (X, 58.7 MB, fits in L2: the apply pass may re-read it there)"},
             "group128_quant": {"ms": k_ms["group128_quant"],
                                "GB/s": bytes_group128() / (k_ms["group128_quant"] * 1e-3) / 1e9},
         }
+        kernels["per_tensor_quant"]["frac_hbm"] = kernels["per_tensor_quant"]["GB/s"] / hbm
+        kernels["per_tensor_quant"]["frac_hbm_unique"] = kernels["per_tensor_quant"]["GB/s_unique"] / hbm
+        kernels["group128_quant"]["frac_hbm"] = kernels["group128_quant"]["GB/s"] / hbm
+        timed_s = ms * 1e-3
+        bf16_peak = peaks["bf16_tflops"] if timed_s < 5.0 else peaks["bf16_tflops_sustained"]
+        fp8_peak = bf16_peak * FP8_OVER_BF16
         for n in NS:
             t = k_ms[f"gemm_N{n}"]
             kernels[f"gemm_N{n}"] = {"ms": t, "TFLOP/s": 2.0 * M * n * K / (t * 1e-3) / 1e12,
                                      "GB/s": bytes_gemm(M, n) / (t * 1e-3) / 1e9}
-        for kname in ("per_tensor_quant", "group128_quant"):
-            kernels[kname]["frac_hbm"] = kernels[kname]["GB/s"] / peaks["hbm_gbs"]
-        timed_s = ms * 1e-3
-        bf16_peak = peaks["bf16_tflops"] if timed_s < 5.0 else peaks["bf16_tflops_sustained"]
-        fp8_peak = bf16_peak * FP8_OVER_BF16
+            kernels[f"gemm_N{n}"]["frac_fp8"] = kernels[f"gemm_N{n}"]["TFLOP/s"] / fp8_peak
+            if fp8_meas:
+                kernels[f"gemm_N{n}"]["frac_fp8_measured"] = kernels[f"gemm_N{n}"]["TFLOP/s"] / fp8_meas
         # dominant kernel: the block GEMM (sum over the three N per step)
         gemm_ms = sum(k_ms[f"gemm_N{n}"] for n in NS)
         achieved = gemm_flops() / (gemm_ms * 1e-3) / 1e12
-        for n in NS:
-            kernels[f"gemm_N{n}"]["frac_fp8"] = kernels[f"gemm_N{n}"]["TFLOP/s"] / fp8_peak
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": fp8_peak,
+                    "unit": "TFLOP/s", "frac": achieved / fp8_peak,
+                    "traffic": gemm_traffic(),
+                    "traffic_unit": "bytes per GEMM launch (mean of the step's 3), ncu",
+                    "algorithmic_bytes_per_launch": sum(bytes_gemm(M, n) for n in NS) / len(NS),
+                    "kernel": "block_gemm_kernel (all three N per step; at N=7168 the call's "
+                              "time includes tail_reduce_kernel, which sums the split last wave)",
+                    "peak_source": f"{peak_src} bf16 "
+                                   f"{'burst' if timed_s < 5.0 else 'sustained'} x {FP8_OVER_BF16} (fp8/bf16 nominal)"}
+        if fp8_meas:
+            roofline["peak_fp8_measured"] = fp8_meas
+            roofline["frac_fp8_measured"] = achieved / fp8_meas
+            roofline["peak_fp8_measured_source"] = ("cuBLASLt per-tensor FP8 GEMM (torch._scaled_mm, E4M3, "
+                                                    "bf16 out) 8192^3 on random data, best of 10, this process")
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
@@ -435,35 +732,65 @@ def our_arm(args, rank, world, local_rank):
                        "parallelism": f"dp{world}" if world > 1 else "none",
                        "l2": "inputs larger than L2 (X 58.7 MB + weights 360 MB per step)"},
             "kernels": kernels,
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": fp8_peak,
-                         "unit": "TFLOP/s", "frac": achieved / fp8_peak,
-                         "traffic": gemm_traffic(),
-                         "traffic_unit": "bytes per GEMM launch (mean of the step's 3), ncu",
-                         "algorithmic_bytes_per_launch": sum(bytes_gemm(M, n) for n in NS) / len(NS),
-                         "kernel": "block_gemm_kernel (all three N per step; at N=7168 the call's "
-                                   "time includes tail_reduce_kernel, which sums the split last wave)",
-                         "peak_source": f"{peak_src} bf16 "
-                                        f"{'burst' if timed_s < 5.0 else 'sustained'} x {FP8_OVER_BF16} (fp8/bf16 nominal)"},
+            "roofline": roofline,
             "e2e": {"value": total_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
             "gpu_launches": int(launches),
             "clocks": clk,
         }
+        if sharded_ms is not None:
+            rows = M * world
+            result["per_tensor_sharded"] = {
+                "ms": sharded_ms, "rows_total": rows, "K": K,
+                "GB/s_total": bytes_per_tensor(rows, K) / (sharded_ms * 1e-3) / 1e9,
+                "what": "row-sharded per-tensor quant: local amax, one 4-byte NCCL MAX all-reduce, "
+                        "local apply; each rank's X[4096,7168] is its shard; max over ranks"}
+        if table is not None:
+            result["workloads"] = table
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
     return result
 
 
+def single_op(args):
+    """--op: one operation at one shape, one JSON line per timing mode."""
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    import fp8_dynamic_quantization_b200 as fq
+    fq.library()
+    peaks, _ = load_peaks()
+    timer = Timer(dev)
+    n = args.n or 0
+    k = args.k or (2048 if args.op in ("per_tensor", "amax") else 7168)
+    for rec in time_op(timer, args.op, args.m, n, k, dev, args.modes.split(","), args.reps,
+                       peaks["hbm_gbs"], peaks["bf16_tflops"] * FP8_OVER_BF16):
+        print(json.dumps(rec), flush=True)
+    if fq.device_status() != 0:
+        raise SystemExit("device-side error recorded")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-kernels", action="store_true",
+                    help="skip the per-workload kernel table (and the FP8 peak)")
+    ap.add_argument("--op", choices=["per_tensor", "amax", "group128", "group128_ue8m0", "per_channel",
+                                     "gemm", "gemm_pt", "gemm_pc", "gemm_ue8m0", "linear"])
+    ap.add_argument("--m", type=int)
+    ap.add_argument("--n", type=int)
+    ap.add_argument("--k", type=int)
+    ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--modes", default="cold,graph")
     args = ap.parse_args()
+    if args.op:
+        single_op(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))
