@@ -112,6 +112,19 @@ __device__ __forceinline__ uint32_t zero_pair(uint32_t w) {
     return ((w >> 8) & 0x80u) | ((w >> 16) & 0x8000u);
 }
 
+// Codes of 8 bf16 values for a scale in the reciprocal-corrected range
+// (Scale::mode == 1) and values no larger than the amax.
+__device__ __forceinline__ uint2 quant8_fast(const uint4& v, const Scale& d) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(div_fast(bf16_lo(w[i]), d), div_fast(bf16_hi(w[i]), d));
+    uint2 r;
+    r.x = c[0] | (c[1] << 16);
+    r.y = c[2] | (c[3] << 16);
+    return r;
+}
+
 // Codes of 8 bf16 values (one 16-byte vector) -> 8 bytes.  `exact` forces
 // the IEEE division (for values that may exceed the amax).
 __device__ __forceinline__ uint2 quant8(const uint4& v, const Scale& d, bool exact = false) {

@@ -118,8 +118,8 @@ struct GemmCfg {
     static constexpr int kThreads = 128 + 128 * kEpiWG;
     // Register split (setmaxnreg) between warpgroup 0 and the promotion
     // warpgroups; it must add up to at most threads x launch registers.
-    static constexpr int kRegWG0 = kEpiWG == 2 ? (kCW == 128 ? 48 : 56) : 32;
-    static constexpr int kRegEpi = kEpiWG == 2 ? (kCW == 128 ? 224 : 216) : 160;
+    static constexpr int kRegWG0 = kEpiWG == 2 ? (kCW == 128 ? 40 : 56) : 32;
+    static constexpr int kRegEpi = kEpiWG == 2 ? (kCW == 128 ? 232 : 216) : 160;
     static constexpr int kLaunchRegs = ((65536 / kThreads) / 8) * 8 > 255 ? 255 : ((65536 / kThreads) / 8) * 8;
     static_assert(kEpiWG == 1 || 128 * kRegWG0 + 128 * kEpiWG * kRegEpi <= kThreads * kLaunchRegs,
                   "register split exceeds the launch allocation");
@@ -307,6 +307,14 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     constexpr bool PT = C::PT, MX = C::MX, PC = C::PC;
     constexpr bool ONE = PT || MX || PC;  // one TMEM accumulation per unit, no per-K-block promotion
     constexpr int NB = C::kNumBuf;
+    // Per-K-block promotion (block scales): the MMA's commit to empty[s]
+    // also tells the promotion warps that K block `it`'s partial is in TMEM,
+    // and the promotion warps hand a TMEM buffer back by arriving on the
+    // full barrier of the K block that will reuse it (it + NB).  So the
+    // MMA thread waits once and commits once per K block.
+    constexpr bool MERGED = !ONE;
+    constexpr uint32_t kRelease = (PAIR ? 2u : 1u) * 4u * C::kEpiWG;   // promotion warps arriving per release
+    static_assert(!MERGED || NB <= STAGES, "a TMEM buffer is reused within the stage ring");
     constexpr uint32_t kSlots = C::kScaleSlots > 0 ? C::kScaleSlots : 1;   // divisor for the (SS) slot ring
     constexpr uint32_t kSfN = C::kSfSlots > 0 ? C::kSfSlots : 1;         // divisor for the (MX) slot ring
     extern __shared__ uint8_t smem_raw[];
@@ -337,7 +345,13 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     const int unit_step = PAIR ? int(ptx::num_clusters_x()) : int(gridDim.x);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) { ptx::mbar_init(&full[s], 1); ptx::mbar_init(&empty[s], 1); }
+        for (int s = 0; s < STAGES; ++s) {
+            ptx::mbar_init(&full[s], MERGED ? 1 + kRelease : 1);
+            ptx::mbar_init(&empty[s], 1);
+        }
+        if (MERGED)              // the first NB K blocks find their TMEM buffer free
+            for (int j = 0; j < NB; ++j)
+                for (uint32_t a = 0; a < kRelease; ++a) ptx::mbar_arrive(&full[j]);
         for (int b = 0; b < NB; ++b) {
             ptx::mbar_init(&tfull[b], 1);
             ptx::mbar_init(&tempty[b], (PAIR ? 2 : 1) * 4 * C::kEpiWG);
@@ -494,9 +508,11 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 int kb = kb0;
                 for (int st = 0; st < steps && !failed; ++st, ++c) {
                     const uint32_t buf = c % NB, tph = (c / NB) & 1;
-                    const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1, p.wait_budget)
-                                            : ptx::mbar_wait(&tempty[buf], tph ^ 1, p.wait_budget);
-                    if (!freed) { fail(); failed = true; break; }
+                    if (!MERGED) {          // merged: the full wait below covers the buffer
+                        const bool freed = PAIR ? ptx::mbar_wait_cluster(&tempty[buf], tph ^ 1, p.wait_budget)
+                                                : ptx::mbar_wait(&tempty[buf], tph ^ 1, p.wait_budget);
+                        if (!freed) { fail(); failed = true; break; }
+                    }
                     const uint32_t d = tmem_base + buf * BN;
                     const int kb_end = ONE ? kb1 : kb + 1;
                     for (; kb < kb_end; ++kb, ++it) {
@@ -547,6 +563,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                         last_parity = ph;
                     }
                     if (failed) break;
+                    if (MERGED) continue;                                    // empty[s] said it
                     if (PAIR) {                                              // step ready, in both CTAs
                         const uint32_t f0 = ptx::smem_u32(&tfull[buf]);
                         ptx::mma_commit_pair(f0);
@@ -574,8 +591,9 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         uint32_t c = 0;
         uint32_t sg = 0;                          // scale groups consumed (SS)
         uint64_t acc2[C::kCW / 2];
-        // the leader's tempty barriers, as cluster addresses (pair mode)
+        // the leader's tempty (merged: full) barriers, as cluster addresses (pair mode)
         const uint32_t tempty0 = PAIR ? ptx::mapa_shared(ptx::smem_u32(tempty), 0) : 0u;
+        const uint32_t full0 = PAIR ? ptx::mapa_shared(ptx::smem_u32(full), 0) : 0u;
         for (int u = unit0; u < p.units; u += unit_step) {
             int tp, tq, kb0, kb1;
             unit_coords(p, u, tp, tq, kb0, kb1);
@@ -658,33 +676,56 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                 }
                 const uint64_t s2 = ptx::pack_f32x2(s, s);
                 const uint32_t buf = c % NB, tph = (c / NB) & 1;
-                if (!ptx::mbar_wait(&tfull[buf], tph, p.wait_budget)) { fail(); ok = false; break; }
+                const bool landed = MERGED ? ptx::mbar_wait(&empty[c % STAGES], (c / STAGES) & 1, p.wait_budget)
+                                           : ptx::mbar_wait(&tfull[buf], tph, p.wait_budget);
+                if (!landed) { fail(); ok = false; break; }
                 ptx::tc_fence_after();
                 const uint32_t taddr = tmem_base + (uint32_t(quarter * 32) << 16)
                                        + buf * BN + chalf * C::kCW;
                 const float* sl = slab + (kb - kb0) * BN + chalf * C::kCW;
-                // Loads of this thread's kCW columns in chunks of at most 64;
-                // the TMEM buffer is released as soon as the last chunk has
-                // landed, then that chunk's FMAs run.
-                constexpr int kChunk = C::kCW >= 64 ? 64 : C::kCW;
-                constexpr int kChunks = C::kCW / kChunk;
-                float v[kChunk];
-#pragma unroll
-                for (int ch = 0; ch < kChunks; ++ch) {
-                    if constexpr (kChunk == 64) ptx::tmem_ld64(taddr + ch * 64, v);
-                    else if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + ch * 32, v);
-                    else ptx::tmem_ld16(taddr + ch * 16, v);
-                    ptx::tmem_wait_ld();
-                    if (ch == kChunks - 1) {
-                        ptx::tc_fence_before();
-                        __syncwarp();
-                        if (lane == 0) {
-                            if (PAIR) ptx::mbar_arrive_cluster(tempty0 + buf * 8);
-                            else ptx::mbar_arrive(&tempty[buf]);
-                        }
+                // Hand the TMEM buffer back (all of this warp's loads have landed).
+                auto release = [&]() {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        const uint32_t j = (c + NB) % STAGES;           // merged: the K block reusing it
+                        if (MERGED && PAIR) ptx::mbar_arrive_cluster(full0 + j * 8);
+                        else if (MERGED) ptx::mbar_arrive(&full[j]);
+                        else if (PAIR) ptx::mbar_arrive_cluster(tempty0 + buf * 8);
+                        else ptx::mbar_arrive(&tempty[buf]);
                     }
-                    if (SWAP && SM == 0) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
-                    else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
+                };
+                if constexpr (C::kCW == 128) {
+                    // 128 columns: 48, then 80 -- the fewest FMAs between
+                    // the first load and the release that the registers
+                    // (128 accumulators + 80 loaded values) allow
+                    float v[80];
+                    ptx::tmem_ld32(taddr, v);
+                    ptx::tmem_ld16(taddr + 32, v + 32);
+                    ptx::tmem_wait_ld();
+                    fma_uniform<48>(acc2, v, s2);
+                    ptx::tmem_ld64(taddr + 48, v);
+                    ptx::tmem_ld16(taddr + 112, v + 64);
+                    ptx::tmem_wait_ld();
+                    release();
+                    fma_uniform<80>(acc2 + 24, v, s2);
+                } else {
+                    // Loads of this thread's kCW columns in chunks of at most 64;
+                    // the TMEM buffer is released as soon as the last chunk has
+                    // landed, then that chunk's FMAs run.
+                    constexpr int kChunk = C::kCW >= 64 ? 64 : C::kCW;
+                    constexpr int kChunks = C::kCW / kChunk;
+                    float v[kChunk];
+#pragma unroll
+                    for (int ch = 0; ch < kChunks; ++ch) {
+                        if constexpr (kChunk == 64) ptx::tmem_ld64(taddr + ch * 64, v);
+                        else if constexpr (kChunk == 32) ptx::tmem_ld32(taddr + ch * 32, v);
+                        else ptx::tmem_ld16(taddr + ch * 16, v);
+                        ptx::tmem_wait_ld();
+                        if (ch == kChunks - 1) release();
+                        if (SWAP && SM == 0) fma_columns<kChunk>(acc2 + ch * kChunk / 2, v, sl + ch * kChunk);
+                        else fma_uniform<kChunk>(acc2 + ch * kChunk / 2, v, s2);
+                    }
                 }
             }
             if (!ok) break;
