@@ -224,7 +224,11 @@ class Timer:
            `reps` calls.
     graph: `reps` calls captured in one CUDA graph and replayed; time / reps
            (how the pages timed their amax kernel; inputs that fit in L2 stay
-           L2-warm)."""
+           L2-warm).
+    stream: like graph, but the calls cycle over several copies of the
+           inputs whose total exceeds L2, so every call reads its input from
+           HBM while its launch overlaps the previous call as in a step (no
+           event or host gap between calls)."""
 
     def __init__(self, dev):
         self.dev = dev
@@ -246,27 +250,37 @@ class Timer:
         return statistics.median(ts)
 
     def graph(self, fn, reps):
-        fn()
+        return self.stream([fn], reps)
+
+    def stream(self, fns, reps, replays=1):
+        """Graph of `reps` calls cycling over `fns`; time per call (median
+        of `replays` replays)."""
+        for fn in fns:
+            fn()
         torch.cuda.synchronize()
         s = torch.cuda.Stream()
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            fn()                      # populate per-stream workspace caches
+            for fn in fns:
+                fn()                  # populate per-stream workspace caches
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=s):
-            for _ in range(reps):
-                fn()
+            for i in range(reps):
+                fns[i % len(fns)]()
         g.replay()
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        g.replay()
-        b.record()
-        b.synchronize()
+        ts = []
+        for _ in range(replays):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            g.replay()
+            b.record()
+            b.synchronize()
+            ts.append(a.elapsed_time(b) * 1e3 / reps)
         del g
-        return a.elapsed_time(b) * 1e3 / reps
+        return statistics.median(ts)
 
 
 # ---------------------------------------------------------------- operations
@@ -283,33 +297,45 @@ def _out(m, n, dev):
     return torch.empty(m, (n + 7) // 8 * 8, dtype=torch.bfloat16, device=dev)[:, :n]
 
 
-def make_op(op, m, n, k, dev):
-    """(callable, algorithmic bytes, flops or None, extra record fields) for
-    one operation at one shape, on seeded synthetic inputs of its workload."""
+def input_copies(nbytes):
+    """Copies of an input that together exceed L2 twice over (at least 2,
+    at most 8), for the rotating `stream` timing."""
+    return int(min(8, max(2, -(-2 * L2_BYTES // max(1, int(nbytes))))))
+
+
+def make_op(op, m, n, k, dev, copies=1):
+    """(callables, algorithmic bytes, flops or None, extra record fields) for
+    one operation at one shape, on seeded synthetic inputs of its workload.
+    The quantisation ops get `copies` callables, each on its own copy of the
+    input (the others get one)."""
     import fp8_dynamic_quantization_b200 as fq
+
+    def xs(x):
+        x = x.to(dev)
+        return [x] + [x.clone() for _ in range(copies - 1)]
     if op == "per_tensor":
-        x = inputs.activations_per_tensor(m, k=k).to(dev)
-        return (lambda: fq.act_quant_per_tensor(x)), bytes_per_tensor(m, k), None, {
-            "GB/s_basis": "5 B/element (amax read + apply read + code write)",
-            "unique_bytes": bytes_per_tensor(m, k, unique=True)}
+        return [(lambda x=x: fq.act_quant_per_tensor(x)) for x in xs(inputs.activations_per_tensor(m, k=k))], \
+            bytes_per_tensor(m, k), None, {
+                "GB/s_basis": "5 B/element (amax read + apply read + code write)",
+                "unique_bytes": bytes_per_tensor(m, k, unique=True)}
     if op == "amax":
-        x = inputs.activations_per_tensor(m, k=k).to(dev)
-        return (lambda: fq.act_amax(x)), bytes_amax(m, k), None, {}
+        return [(lambda x=x: fq.act_amax(x)) for x in xs(inputs.activations_per_tensor(m, k=k))], \
+            bytes_amax(m, k), None, {}
     if op == "group128":
-        x = inputs.activations_group(m, k=k).to(dev)
-        return (lambda: fq.act_quant_group128(x)), bytes_group128(m, k), None, {}
+        return [(lambda x=x: fq.act_quant_group128(x)) for x in xs(inputs.activations_group(m, k=k))], \
+            bytes_group128(m, k), None, {}
     if op == "group128_ue8m0":
-        x = inputs.activations_group(m, k=k).to(dev)
-        return (lambda: fq.act_quant_group128_ue8m0(x)), 3.0 * m * k + m * (k // 128), None, {}
+        return [(lambda x=x: fq.act_quant_group128_ue8m0(x)) for x in xs(inputs.activations_group(m, k=k))], \
+            3.0 * m * k + m * (k // 128), None, {}
     if op == "per_channel":
-        x = inputs.activations_per_tensor(m, k=k).to(dev)
-        return (lambda: fq.act_quant_per_channel(x)), 3.0 * m * k + 4.0 * m, None, {}
+        return [(lambda x=x: fq.act_quant_per_channel(x)) for x in xs(inputs.activations_per_tensor(m, k=k))], \
+            3.0 * m * k + 4.0 * m, None, {}
     flops = 2.0 * m * n * k
     if op == "gemm":
         qa, sa, qb, sb = inputs.gemm_operands(m, n, k)
         tqa, tqb, tsa, tsb = _dev_codes(qa, dev), _dev_codes(qb, dev), _dev(sa, dev), _dev(sb, dev)
         y = _out(m, n, dev)
-        return (lambda: fq.block_gemm(tqa, tsa, tqb, tsb, out=y)), bytes_gemm(m, n, k), flops, {}
+        return [lambda: fq.block_gemm(tqa, tsa, tqb, tsb, out=y)], bytes_gemm(m, n, k), flops, {}
     if op in ("gemm_pt", "gemm_pc", "gemm_ue8m0"):
         qa, _, qb, _ = inputs.gemm_operands(m, n, k)
         tqa, tqb = _dev_codes(qa, dev), _dev_codes(qb, dev)
@@ -317,16 +343,16 @@ def make_op(op, m, n, k, dev):
         g = inputs.rng(m + n)
         if op == "gemm_pt":
             sa, sb = torch.tensor([0.01], device=dev), torch.tensor([0.02], device=dev)
-            return (lambda: fq.gemm_per_tensor(tqa, sa, tqb, sb, out=y)), \
+            return [lambda: fq.gemm_per_tensor(tqa, sa, tqb, sb, out=y)], \
                 m * k + n * k + 8.0 + 2.0 * m * n, flops, {}
         if op == "gemm_pc":
             sa = _dev(g.uniform(1e-3, 1e-1, m).astype(np.float32), dev)
             sb = _dev(g.uniform(1e-3, 1e-1, n).astype(np.float32), dev)
-            return (lambda: fq.gemm_per_channel(tqa, sa, tqb, sb, out=y)), \
+            return [lambda: fq.gemm_per_channel(tqa, sa, tqb, sb, out=y)], \
                 m * k + n * k + 4.0 * (m + n) + 2.0 * m * n, flops, {}
         sa = _dev(g.integers(115, 135, (m, k // 128)).astype(np.uint8), dev)
         sb = _dev(g.integers(115, 135, ((n + 127) // 128, k // 128)).astype(np.uint8), dev)
-        return (lambda: fq.block_gemm_ue8m0(tqa, sa, tqb, sb, out=y)), \
+        return [lambda: fq.block_gemm_ue8m0(tqa, sa, tqb, sb, out=y)], \
             m * k + n * k + m * k / 128 + ((n + 127) // 128) * k / 128 + 2.0 * m * n, flops, {}
     if op == "linear":
         # the one-call group-128 linear: quantisation kernel, then the GEMM
@@ -335,16 +361,22 @@ def make_op(op, m, n, k, dev):
         qb, sb = inputs.weight_operands(n, k)
         tqb, tsb = _dev_codes(qb, dev), _dev(sb, dev)
         y = _out(m, n, dev)
-        return (lambda: fq.linear_fused(x, tqb, tsb, out=y)), \
+        return [lambda: fq.linear_fused(x, tqb, tsb, out=y)], \
             2.0 * m * k + n * k + 4.0 * ((n + 127) // 128) * (k // 128) + 2.0 * m * n, flops, {}
     raise ValueError(op)
 
 
+QUANT_OPS = ("per_tensor", "amax", "group128", "group128_ue8m0", "per_channel")
+
+
 def time_op(timer, op, m, n, k, dev, modes, reps, hbm, fp8_peak):
-    fn, nbytes, flops, extra = make_op(op, m, n, k, dev)
+    copies = input_copies(2.0 * m * k) if (op in QUANT_OPS and "stream" in modes) else 1
+    fns, nbytes, flops, extra = make_op(op, m, n, k, dev, copies)
     out = []
     for mode in modes:
-        us = getattr(timer, mode)(fn, reps)
+        if mode == "stream" and op not in QUANT_OPS:
+            continue
+        us = timer.stream(fns, reps, replays=3) if mode == "stream" else getattr(timer, mode)(fns[0], reps)
         rec = {"op": op, "M": m, "N": n, "K": k, "mode": mode, "us": us,
                "GB/s": nbytes / us / 1e3, "frac_hbm": nbytes / us / 1e3 / hbm}
         if "unique_bytes" in extra:
@@ -353,8 +385,10 @@ def time_op(timer, op, m, n, k, dev, modes, reps, hbm, fp8_peak):
         if flops:
             rec["TFLOP/s"] = flops / us / 1e6
             rec["frac_fp8"] = flops / us / 1e6 / fp8_peak
+        if mode == "stream":
+            rec["input_copies"] = copies
         out.append(rec)
-    del fn
+    del fns
     return out
 
 
@@ -392,7 +426,7 @@ def workload_table(dev, hbm, fp8_peak, reps=20):
     rows = []
 
     def add(op, m, n, k, big):
-        modes = ["graph", "cold"] if big else ["graph"]
+        modes = ["graph", "cold", "stream"] if big else ["graph"]
         rows.extend(time_op(timer, op, m, n, k, dev, modes, reps, hbm, fp8_peak))
     # workload 1: the tiny linear layer
     add("per_tensor", 64, 0, 2048, False)
@@ -587,6 +621,26 @@ def our_arm(args, rank, world, local_rank):
     k_ms = {"per_tensor_quant": avg(0, 1), "group128_quant": avg(1, 2)}
     for i, n in enumerate(NS):
         k_ms[f"gemm_N{n}"] = avg(2 + i, 3 + i)
+    # What an event pair costs by itself: the same bracketing around an
+    # empty kernel.
+    floor_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(50)]
+    for a, b in floor_ev:
+        a.record(stream)
+        torch.cuda._sleep(0)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    event_floor_ms = statistics.median(a.elapsed_time(b) for a, b in floor_ev)
+    # The quantisation kernels back to back as in the step (launches
+    # overlapping, no events between them) on copies of X that together
+    # exceed L2, so every call reads its X from HBM.
+    timer = Timer(dev)
+    x_copies = [x] + [x.clone() for _ in range(input_copies(x.numel() * 2) - 1)]
+    pipe_ms = {
+        "per_tensor_quant": timer.stream([(lambda t=t: fq.act_quant_per_tensor(t)) for t in x_copies],
+                                         40, replays=5) * 1e-3,
+        "group128_quant": timer.stream([(lambda t=t: fq.act_quant_group128(t)) for t in x_copies],
+                                       40, replays=5) * 1e-3}
+    del timer, x_copies
 
     if dist is not None:
         t = torch.tensor([ms], dtype=torch.float64, device=dev)
@@ -679,19 +733,24 @@ def our_arm(args, rank, world, local_rank):
         total_flops = gemm_flops() * world
         value = total_flops / (step_ms * 1e-3) / 1e12
         hbm = peaks["hbm_gbs"]
-        t_pt = k_ms["per_tensor_quant"]
+        t_pt = pipe_ms["per_tensor_quant"]
+        t_g = pipe_ms["group128_quant"]
         kernels = {
-            "timing": "per-kernel: in-stream events between the calls of a second pass over the same "
-                      "steps; sum of these can exceed ms_per_step (the events stop each launch from "
-                      "overlapping the previous kernel's tail)",
+            "timing": "GEMMs: in-stream events between the calls of a second pass over the same steps. "
+                      "Quantisation kernels (ms): the kernel alone back to back as in the step, launches "
+                      "overlapping, on copies of X that together exceed L2 (each call reads its X from "
+                      "HBM); ms_with_events: the second pass's event pair around the call, which also "
+                      "holds the event pair's own cost (event_floor_ms, measured around an empty kernel)",
+            "event_floor_ms": event_floor_ms,
             "per_tensor_quant": {
                 "ms": t_pt,
+                "ms_with_events": k_ms["per_tensor_quant"],
                 "GB/s": bytes_per_tensor() / (t_pt * 1e-3) / 1e9,
                 "GB/s_unique": bytes_per_tensor(unique=True) / (t_pt * 1e-3) / 1e9,
                 "basis": "GB/s at 5 B/element (amax read, apply read, code write); GB/s_unique at "
                          "3 B/element (X, 58.7 MB, fits in L2: the apply pass may re-read it there)"},
-            "group128_quant": {"ms": k_ms["group128_quant"],
-                               "GB/s": bytes_group128() / (k_ms["group128_quant"] * 1e-3) / 1e9},
+            "group128_quant": {"ms": t_g, "ms_with_events": k_ms["group128_quant"],
+                               "GB/s": bytes_group128() / (t_g * 1e-3) / 1e9},
         }
         kernels["per_tensor_quant"]["frac_hbm"] = kernels["per_tensor_quant"]["GB/s"] / hbm
         kernels["per_tensor_quant"]["frac_hbm_unique"] = kernels["per_tensor_quant"]["GB/s_unique"] / hbm

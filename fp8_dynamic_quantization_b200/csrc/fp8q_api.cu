@@ -42,7 +42,14 @@ struct DeviceInfo {
     int status = FP8Q_OK;
     int sms = 0;
     int index = 0;
+    int64_t l2_bytes = 0;
 };
+
+// The per-tensor passes hold a tensor of at most half the L2 there between
+// the amax pass and the apply pass (measured at 4096 x 7168, 58.7 MB of a
+// 126 MB L2: 26.3 against 28.2 us per call; at 16384 x 7168, above L2, the
+// same hints cost 3%).
+bool keep_in_l2(const DeviceInfo* d, int64_t bytes) { return bytes <= d->l2_bytes / 2; }
 
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -123,6 +130,7 @@ int device_info(DeviceInfo** out) {
             d.index = dev;
             if (prop.major != 10) d.status = FP8Q_ERR_NO_DEVICE;
             d.sms = prop.multiProcessorCount;
+            d.l2_bytes = prop.l2CacheSize;
             if (d.status == FP8Q_OK) {
                 cudaError_t e = cudaSuccess;
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12>();
@@ -240,7 +248,7 @@ const TableRow kGemmTable[] = {
 struct GemmPlan {
     bool swap, pair;
     int bn, stages, splits, tiles_p, tiles_q, units, grid;
-    int full_tiles, tail_tiles, tail_splits;   // split tail (normal tiles only)
+    int full_tiles, tail_tiles, tail_splits;   // split tail (normal and pair tiles)
     int64_t ldw;
     size_t ws_bytes;
 };
@@ -300,8 +308,8 @@ bool tile_override(TableRow* out) {
     return has;
 }
 
-// Only the fp32 block-scaled GEMM has a CTA-pair variant: for the others a
-// forced pair row runs as the single-CTA tile of the same width.
+// no_pair: a pair row runs as the single-CTA tile of the same width (the
+// scale modes other than fp32 block scales).
 //
 // Split tail: with one whole tile per unit, a tile count just above a
 // multiple of the SM count leaves a last wave in which few SMs work for a
@@ -352,10 +360,11 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
     pl.full_tiles = int(tiles);
     pl.tail_tiles = 0;
     pl.tail_splits = 1;
-    if (!pl.swap && !pl.pair && splits == 1 && tiles > sms && tiles % sms != 0) {
-        const int tail = int(tiles % sms);
-        const size_t slot_bytes = size_t(tail) * 128 * size_t(pl.bn) * sizeof(float);   // one split of every tail tile
-        const int s = int(std::min<size_t>(size_t(std::min(sms / tail, G / 2)), ws_cap / slot_bytes));
+    const int slots = pl.pair ? sms / 2 : sms;          // tiles that run at once
+    if (!pl.swap && splits == 1 && tiles > slots && tiles % slots != 0) {
+        const int tail = int(tiles % slots);
+        const size_t slot_bytes = size_t(tail) * tile_rows * size_t(pl.bn) * sizeof(float);   // one split of every tail tile
+        const int s = int(std::min<size_t>(size_t(std::min(slots / tail, G / 2)), ws_cap / slot_bytes));
         if (s >= 2) {
             pl.tail_tiles = tail;
             pl.tail_splits = s;
@@ -367,7 +376,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
                       : std::max(1, std::min(pl.units, sms));
     pl.ldw = (N + 7) / 8 * 8;
     pl.ws_bytes = splits > 1 ? size_t(splits) * size_t(M) * size_t(pl.ldw) * sizeof(float)
-                : pl.tail_tiles > 0 ? size_t(pl.tail_tiles) * size_t(pl.tail_splits) * 128 * size_t(pl.bn) * sizeof(float)
+                : pl.tail_tiles > 0 ? size_t(pl.tail_tiles) * size_t(pl.tail_splits) * tile_rows * size_t(pl.bn) * sizeof(float)
                 : 0;
     return pl;
 }
@@ -481,8 +490,8 @@ const char* fp8q_status_string(int status) {
 
 int fp8q_abi_version(void) { return (1 << 16) | 1; }
 
-// Host only: the launch plan fp8_block_gemm (fp32, per-tensor and
-// per-channel scales) would use on a device with `sms` SMs.
+// Host only: the launch plan fp8_block_gemm would use on a device with
+// `sms` SMs (the other scale modes run pair rows as single-CTA tiles).
 int fp8q_gemm_plan(int64_t M, int64_t N, int64_t K, int sms, size_t ws_cap, int* plan, size_t* ws_bytes) {
     if (M <= 0 || N <= 0 || K <= 0 || sms <= 0 || !plan || !ws_bytes) return FP8Q_ERR_INVALID_ARG;
     if (K % 128 || M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
@@ -547,10 +556,21 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
         std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: amax+apply grid=%d\n",
                      (long long)M, (long long)K, grid);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
-    if (contig) {
+    const bool keep = keep_in_l2(d, M * ldx * 2);
+    if (contig && keep) {
+        launch(amax_partial_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials);
+        launch(apply_kernel<kStreamU, true, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials, grid, q, ldq, scale);
+    } else if (contig) {
         launch(amax_partial_kernel<kStreamU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
         launch(apply_kernel<kStreamU, true, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials,
                                                                             grid, q, ldq, scale);
+    } else if (keep) {
+        launch(amax_partial_kernel<kStreamU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials);
+        launch(apply_kernel<kStreamU, false, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials, grid, q, ldq, scale);
     } else {
         launch(amax_partial_kernel<kStreamU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
         launch(apply_kernel<kStreamU, false, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials,
@@ -581,8 +601,15 @@ int fp8_act_amax(const void* x, int64_t M, int64_t K, int64_t ldx, uint32_t* ama
     const int grid = stream_grid(nvec, d->sms);
     uint32_t* partials = static_cast<uint32_t*>(workspace);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
-    if (ldx == K)
+    const bool keep = keep_in_l2(d, M * ldx * 2);      // for an apply call that follows
+    if (ldx == K && keep)
+        launch(amax_partial_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials);
+    else if (ldx == K)
         launch(amax_partial_kernel<kStreamU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
+    else if (keep)
+        launch(amax_partial_kernel<kStreamU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               partials);
     else
         launch(amax_partial_kernel<kStreamU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, partials);
     // Fold the partials into one word: a single CTA over `grid` words.
@@ -607,9 +634,16 @@ int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
     }
     const int grid = stream_grid(nvec, d->sms);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
-    if (ldx == K && ldq == K)
+    const bool keep = keep_in_l2(d, M * ldx * 2);      // an amax call before this one kept x in L2
+    if (ldx == K && ldq == K && keep)
+        launch(apply_kernel<kStreamU, true, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               amax_bits, 1, q, ldq, scale);
+    else if (ldx == K && ldq == K)
         launch(apply_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, amax_bits, 1,
                                                                            q, ldq, scale);
+    else if (keep)
+        launch(apply_kernel<kStreamU, false, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
+               amax_bits, 1, q, ldq, scale);
     else
         launch(apply_kernel<kStreamU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx, amax_bits, 1,
                                                                             q, ldq, scale);
@@ -759,7 +793,9 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2, ws_cap);   // no ue8m0 pairs
+    // CTA pairs for fp32 block scales only: the one-step modes (per-tensor,
+    // per-channel) measured ~5% slower with pairs, and ue8m0 has none
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode != 0, ws_cap);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -880,10 +916,11 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         launch(splitk_reduce_kernel, dim3(g), dim3(256), 0, st, 1u, p.ws, pl.splits, p.M, p.N, pl.ldw, p.y, ldy);
         rc = launch_status();
     } else if (pl.tail_tiles > 0) {
-        const int64_t total = int64_t(pl.tail_tiles) * 128 * (pl.bn / 4);
+        const int tile_rows = pl.pair ? 256 : 128;
+        const int64_t total = int64_t(pl.tail_tiles) * tile_rows * (pl.bn / 4);
         const int g = int(std::max<int64_t>(1, std::min<int64_t>((total + 255) / 256, int64_t(d->sms) * 8)));
         launch(tail_reduce_kernel, dim3(g), dim3(256), 0, st, 1u, p.ws, pl.tail_tiles, pl.tail_splits, pl.full_tiles,
-                                              pl.tiles_p, pl.bn, p.M, p.N, p.y, ldy);
+                                              pl.tiles_p, tile_rows, pl.bn, p.M, p.N, p.y, ldy);
         rc = launch_status();
     }
     return rc;

@@ -42,12 +42,12 @@
 //           is computed once per work unit into shared memory.
 // Split-K: a unit may cover a sub-range of K blocks; its fp32 partial goes
 // to the workspace and splitk_reduce_kernel adds the splits in fixed order.
-// Split tail (normal tiles): when the tiles leave a last wave that would
-// occupy only a few SMs, the first full_tiles tiles run whole and each of
-// the remaining tail tiles is split into tail_splits K ranges, so the last
-// wave is short and fills the SMs; those partials go to the workspace
-// (tile-local [unit][128][BN] fp32) and tail_reduce_kernel adds them in
-// fixed order into Y.
+// Split tail (normal and pair tiles): when the tiles leave a last wave that
+// would occupy only a few SMs, the first full_tiles tiles run whole and each
+// of the remaining tail tiles is split into tail_splits K ranges, so the
+// last wave is short and fills the SMs; those partials go to the workspace
+// (tile-local [unit][tile rows][BN] fp32) and tail_reduce_kernel adds them
+// in fixed order into Y.
 // Programmatic dependent launch: every GEMM is launched as a programmatic
 // dependent of the previous kernel on the stream; its prologue (barriers,
 // TMEM allocation, tensor-map prefetch) overlaps that kernel's tail, and
@@ -93,7 +93,7 @@ struct GemmParams {
     int tiles_p, splits, units;
     int full_units;      // units [0, full_units): tiles x splits; the rest are split-tail units
     int full_tiles;      // tiles before the split tail
-    int tail_splits;     // K ranges per tail tile; their partials go to ws as [unit - full_units][128][BN]
+    int tail_splits;     // K ranges per tail tile; their partials go to ws as [unit - full_units][tile rows][BN]
     // Flags as bytes and no field the kernel does not read: the struct is
     // passed by value to every launch, and growing it from 120 to 136
     // bytes measurably slowed the kernel (2%).
@@ -809,8 +809,8 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     }
                 }
             } else {
-                // fp32 partial: split-K slot [split][M][ldw], or (split tail,
-                // normal tiles) slot u - full_units laid out [128][BN] per tile
+                // fp32 partial: split-K slot [split][M][ldw], or (split tail)
+                // slot u - full_units laid out [tile rows][BN] per tile
                 const bool tail = u >= p.full_units;
                 const int split = u % p.splits;
                 float* wsp = p.ws + int64_t(split) * p.M * p.ldw;
@@ -835,7 +835,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                             const int m = m_base + k;
                             if (m >= p.M) continue;
                             // row m, indexed by the output column n
-                            float* wr = tail ? p.ws + (int64_t(u - p.full_units) * 128 + r_base + k) * BN - q0
+                            float* wr = tail ? p.ws + (int64_t(u - p.full_units) * C::kTileRows + int(rank) * 128 + r_base + k) * BN - q0
                                              : wsp + int64_t(m) * p.ldw;
                             if (n + 4 <= p.N) {
                                 *reinterpret_cast<uint4*>(wr + n) = a[k];
@@ -851,7 +851,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                     const int m = m_row;
                     const int n_first = q0 + chalf * C::kCW;
                     if (m < p.M) {
-                        float* wr = tail ? p.ws + (int64_t(u - p.full_units) * 128 + row) * BN - q0
+                        float* wr = tail ? p.ws + (int64_t(u - p.full_units) * C::kTileRows + int(rank) * 128 + row) * BN - q0
                                          : wsp + int64_t(m) * p.ldw;
 #pragma unroll
                         for (int j = 0; j < C::kCW; j += 4) {
@@ -925,32 +925,33 @@ splitk_reduce_kernel(const float* __restrict__ ws, int splits, int M, int N, int
 }
 
 // Fixed-order sum of the split-tail partials (slot tt * splits + s holds
-// split s of tail tile tt, 128 x bn fp32) and conversion to bf16 into Y.
+// split s of tail tile tt, tile_rows x bn fp32) and conversion to bf16 into Y.
 // Each thread handles 4 consecutive columns of one tile row.
 __global__ void __launch_bounds__(256)
 tail_reduce_kernel(const float* __restrict__ ws, int tail_tiles, int splits, int full_tiles, int tiles_p,
-                   int bn, int M, int N, uint16_t* __restrict__ y, int64_t ldy) {
+                   int tile_rows, int bn, int M, int N, uint16_t* __restrict__ y, int64_t ldy) {
     pdl_begin();
     const int quads = bn / 4;
-    const int64_t per_tile = int64_t(128) * quads;
+    const int64_t per_tile = int64_t(tile_rows) * quads;
     const int64_t total = int64_t(tail_tiles) * per_tile;
+    const int64_t slot = int64_t(tile_rows) * bn;
     for (int64_t i = int64_t(blockIdx.x) * 256 + threadIdx.x; i < total; i += int64_t(gridDim.x) * 256) {
         const int tt = int(i / per_tile);
         const int rem = int(i - int64_t(tt) * per_tile);
         const int r = rem / quads;
         const int c = (rem - r * quads) * 4;
         const int tile = full_tiles + tt;
-        const int64_t m = int64_t(tile % tiles_p) * 128 + r;
+        const int64_t m = int64_t(tile % tiles_p) * tile_rows + r;
         const int n = (tile / tiles_p) * bn + c;
         if (m >= M || n >= N) continue;
-        const float* src = ws + (int64_t(tt) * splits * 128 + r) * bn + c;
+        const float* src = ws + (int64_t(tt) * splits * tile_rows + r) * bn + c;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
         // loads issued 6 at a time, added in split order
         for (int s0 = 0; s0 < splits; s0 += 6) {
             float4 v[6];
 #pragma unroll
             for (int t = 0; t < 6; ++t)
-                v[t] = s0 + t < splits ? __ldcs(reinterpret_cast<const float4*>(src + int64_t(s0 + t) * 128 * bn))
+                v[t] = s0 + t < splits ? __ldcs(reinterpret_cast<const float4*>(src + int64_t(s0 + t) * slot))
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
             for (int t = 0; t < 6; ++t)

@@ -15,7 +15,9 @@
 //                            (or reads one amax word), computes the scale,
 //                            writes codes.  Walks the tensor backwards, so
 //                            the part of x the amax pass read last is still
-//                            in L2 when it is read again.
+//                            in L2 when it is read again; a tensor of at most
+//                            half the L2 is held there whole (evict-last
+//                            reads in the amax pass, evict-first here).
 //  per_tensor_cluster_kernel small tensors: one launch of one thread-block
 //                            cluster; values stay in registers while the
 //                            CTAs exchange partial maxima on chip.
@@ -109,22 +111,25 @@ group128_quant_kernel(const uint16_t* __restrict__ x, int64_t ldx,
 
 // ---------------------------------------------------------------------------
 // Per-tensor amax: partial max per CTA into partials[blockIdx.x].
+// KEEP: the tensor fits in L2 with room to spare; its lines are read
+// evict-last for the apply pass that follows.
 // ---------------------------------------------------------------------------
-template <int U, bool CONTIG>
+template <int U, bool CONTIG, bool KEEP = false>
 __global__ void __launch_bounds__(kQuantThreads)
 amax_partial_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row,
                     int64_t ldx, uint32_t* __restrict__ partials) {
     pdl_begin();
     __shared__ uint32_t red[kQuantThreads / 32];
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
+    const uint64_t pol = KEEP ? l2_policy_evict_last() : 0ull;
     uint32_t m = 0;
     for (int64_t i0 = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x; i0 < nvec; i0 += U * stride) {
         uint4 v[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i = i0 + u * stride;
-            v[u] = (i < nvec) ? ld_stream16(x + vec_offset<CONTIG>(i, vec_per_row, ldx))
-                              : make_uint4(0, 0, 0, 0);
+            const uint16_t* src = x + vec_offset<CONTIG>(i, vec_per_row, ldx);
+            v[u] = (i < nvec) ? (KEEP ? ld_stream16_hint(src, pol) : ld_stream16(src)) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
@@ -137,8 +142,9 @@ amax_partial_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_pe
 // Per-tensor apply: amax = max(partials[0:nparts]); scale; codes.
 // ---------------------------------------------------------------------------
 // CHECK: the amax comes from the caller, so a vector may hold values above
-// it (or Inf); such vectors take the IEEE division.
-template <int U, bool CONTIG, bool CHECK>
+// it (or Inf); such vectors take the IEEE division.  KEEP: the amax pass
+// kept the tensor in L2; read it evict-first (its last use).
+template <int U, bool CONTIG, bool CHECK, bool KEEP = false>
 __global__ void __launch_bounds__(kQuantThreads)
 apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, int64_t ldx,
              const uint32_t* __restrict__ partials, int nparts,
@@ -153,6 +159,7 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
     if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = d.s;
 
     const int64_t stride = int64_t(gridDim.x) * kQuantThreads;
+    const uint64_t pol = KEEP ? l2_policy_evict_first() : 0ull;
     const int64_t span = U * stride;
     const int64_t first = int64_t(blockIdx.x) * kQuantThreads + threadIdx.x;
     const int64_t iters = (nvec + span - 1) / span;
@@ -162,8 +169,8 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
 #pragma unroll
         for (int u = 0; u < U; ++u) {
             const int64_t i = i0 + u * stride;
-            v[u] = (i < nvec) ? ld_stream16(x + vec_offset<CONTIG>(i, vec_per_row, ldx))
-                              : make_uint4(0, 0, 0, 0);
+            const uint16_t* src = x + vec_offset<CONTIG>(i, vec_per_row, ldx);
+            v[u] = (i < nvec) ? (KEEP ? ld_stream16_hint(src, pol) : ld_stream16(src)) : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {

@@ -204,33 +204,36 @@ def test_plan_argument_checks(cuda_lib):
 
 
 def test_plan_prefill_tiles_and_split_last_wave(cuda_lib):
-    # 4096 x 7168: 32 x 28 = 896 tiles of 128 x 256 = 6 waves of 148 + 8;
-    # the 8 are split into min(148 // 8, 56 // 2) = 18 K ranges
+    # 4096 x 7168: CTA pairs, 16 x 28 = 448 tiles of 256 x 256 = 6 waves of
+    # 74 pairs + 4; the 4 are split into min(74 // 4, 56 // 2) = 18 K ranges
     p = gemm_plan(cuda_lib, 4096, 7168, 7168)
-    assert (p["swap"], p["pair"], p["bn"], p["splits"]) == (0, 0, 256, 1)
-    assert (p["tiles_p"], p["tiles_q"], p["tail_tiles"], p["tail_splits"]) == (32, 28, 8, 18)
-    assert p["units"] == 888 + 8 * 18 and p["grid"] == 148
-    assert p["ws"] == 8 * 18 * 128 * 256 * 4
-    # last waves of 84 and 112 tiles hold more than half the SMs: whole tiles
-    for n, tail in ((18432, 84), (24576, 112)):
+    assert (p["swap"], p["pair"], p["bn"], p["splits"]) == (0, 1, 256, 1)
+    assert (p["tiles_p"], p["tiles_q"], p["tail_tiles"], p["tail_splits"]) == (16, 28, 4, 18)
+    assert p["units"] == 444 + 4 * 18 and p["grid"] == 148
+    assert p["ws"] == 4 * 18 * 256 * 256 * 4
+    # last waves of 42 and 56 tiles hold more than half the pairs: whole tiles
+    for n, tail in ((18432, 42), (24576, 56)):
         p = gemm_plan(cuda_lib, 4096, n, 7168)
-        assert (p["tiles_p"] * p["tiles_q"]) % 148 == tail
+        assert p["pair"] == 1 and (p["tiles_p"] * p["tiles_q"]) % 74 == tail
         assert (p["tail_tiles"], p["units"], p["ws"]) == (0, p["tiles_p"] * p["tiles_q"], 0)
 
 
 def test_plan_tile_choice_by_m_and_n(cuda_lib):
     def key(m, n):
         p = gemm_plan(cuda_lib, m, n, 7168)
-        return ("swap" if p["swap"] else "normal", p["bn"])
+        return ("swap" if p["swap"] else "pair" if p["pair"] else "normal", p["bn"])
     assert key(1, 18432) == ("swap", 16) and key(16, 7168) == ("swap", 16)
     assert key(17, 2048) == ("swap", 32) and key(32, 18432) == ("swap", 32)
     for m in (33, 64, 128):
         assert key(m, 2048) == ("normal", 128)
         assert key(m, 7168) == ("normal", 256)
         assert key(m, 18432) == ("normal", 128)
-    for m in (129, 256, 512, 4096):
+    for m in (129, 256, 512):
         for n in (2048, 7168, 18432):
             assert key(m, n) == ("normal", 256)
+    for m in (513, 1024, 4096):
+        for n in (2048, 7168, 18432):
+            assert key(m, n) == ("pair", 256)
 
 
 def test_plan_split_k_fills_the_sms_and_respects_a_cap(cuda_lib):
@@ -247,18 +250,22 @@ def test_plan_split_k_fills_the_sms_and_respects_a_cap(cuda_lib):
 
 
 def test_plan_cap_cuts_the_split_tail_and_the_swapped_minimum(cuda_lib):
-    # 4000 x 7100 x 4608: 896 tiles, tail of 8, 36 K blocks -> 18 ranges,
-    # 18 MiB of partials; under the 8 MiB cap 8 ranges
+    # 4000 x 7100 x 4608: 448 pair tiles, tail of 4, 36 K blocks -> 18 ranges,
+    # 18 MiB of partials; under the 8 MiB cap (1 MiB per range) 8 ranges
     p = gemm_plan(cuda_lib, 4000, 7100, 4608)
-    assert (p["tail_tiles"], p["tail_splits"]) == (8, 18) and p["ws"] > NOALLOC_CAP
+    assert (p["tail_tiles"], p["tail_splits"]) == (4, 18) and p["ws"] > NOALLOC_CAP
     q = gemm_plan(cuda_lib, 4000, 7100, 4608, cap=NOALLOC_CAP)
-    assert (q["tail_tiles"], q["tail_splits"]) == (8, 8) and q["ws"] <= NOALLOC_CAP
+    assert (q["tail_tiles"], q["tail_splits"]) == (4, 8) and q["ws"] <= NOALLOC_CAP
+    # single-CTA tiles (M <= 512): 512 x 7100 x 4608 -> 4 x 28 = 112 tiles, one
+    # wave, nothing to split
+    p = gemm_plan(cuda_lib, 512, 7100, 4608)
+    assert (p["pair"], p["tail_tiles"], p["units"]) == (0, 0, 112)
     # 32 swapped tokens with 65 K blocks need 2 K ranges whatever the cap
     q = gemm_plan(cuda_lib, 32, 32776, 8320, cap=NOALLOC_CAP)
     assert q["swap"] == 1 and q["splits"] == 2 and q["ws"] == 2 * 32 * 32776 * 4 > NOALLOC_CAP
 
 
 def test_plan_depends_on_the_sm_count(cuda_lib):
-    # 4096 x 7168 on 132 SMs: 896 = 6 * 132 + 104 -> more than half a wave
+    # 4096 x 7168 on 132 SMs (66 pairs): 448 = 6 * 66 + 52 -> more than half a wave
     p = gemm_plan(cuda_lib, 4096, 7168, 7168, sms=132)
     assert (p["tail_tiles"], p["grid"]) == (0, 132)

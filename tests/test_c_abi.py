@@ -24,7 +24,7 @@ int main(void) {
     /* arguments are checked on the host before any device is touched */
     if (fp8_act_quant_group128((const void*)0, 4, 128, 128, (uint8_t*)0, 128, (float*)0, (void*)0)
         != FP8Q_ERR_INVALID_ARG) return 5;
-    printf("bn=%d splits=%d tail=%dx%d ws=%zu\n", plan[2], plan[4], plan[9], plan[10], ws);
+    printf("pair=%d bn=%d splits=%d tail=%dx%d ws=%zu\n", plan[1], plan[2], plan[4], plan[9], plan[10], ws);
     return 0;
 }
 """
@@ -40,4 +40,4 @@ def test_plain_c_program_links_and_calls_the_library(cuda_lib, tmp_path):
                     "-L", PKG, "-l:libfp8q.so", f"-Wl,-rpath,{PKG}"], check=True)
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
-    assert out.stdout.strip() == f"bn=256 splits=1 tail=8x18 ws={8 * 18 * 128 * 256 * 4}"
+    assert out.stdout.strip() == f"pair=1 bn=256 splits=1 tail=4x18 ws={4 * 18 * 256 * 256 * 4}"

@@ -18,7 +18,8 @@ import oracle
 import fp8_dynamic_quantization_b200 as fq
 from fp8_dynamic_quantization_b200 import inputs
 dev = torch.device("cuda:0")
-for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 256)]:
+shapes = [tuple(int(v) for v in s.split("x")) for s in sys.argv[3].split(",")]
+for m, n, k in shapes:
     qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m + n + k)
     y = fq.block_gemm(torch.from_numpy(qa).to(dev), torch.from_numpy(sa).to(dev),
                       torch.from_numpy(qb).to(dev), torch.from_numpy(sb).to(dev))
@@ -26,7 +27,7 @@ for m, n, k in [(1, 200, 256), (130, 300, 512), (600, 520, 1280), (1025, 264, 25
     Y = y.float().cpu().numpy().astype(np.float64)
     bad = int((np.abs(Y - R) > oracle.gemm_tolerance(R, T)).sum())
     assert bad == 0, (m, n, k, bad)
-    # per-tensor scales; a forced pair row runs it as the single-CTA tile
+    # per-tensor scales (pair rows run the pair kernel here too)
     s_a, s_b = np.float32(0.05), np.float32(0.003)
     y = fq.gemm_per_tensor(torch.from_numpy(qa).to(dev), torch.tensor([s_a], device=dev),
                            torch.from_numpy(qb).to(dev), torch.tensor([s_b], device=dev))
@@ -58,10 +59,25 @@ print("ok")
 '''
 
 
+def _run_child(tile, shapes):
+    env = dict(os.environ, FP8Q_GEMM_TILE=tile)
+    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, tile, shapes], env=env, capture_output=True,
+                       text=True, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+
+
 @pytest.mark.parametrize("tile", ["normal:128", "normal:192", "normal:256", "pair:256", "pair:128",
                                   "swap:16", "swap:32", "swap:64", "swap:128:3"])
 def test_gemm_mode_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
-    env = dict(os.environ, FP8Q_GEMM_TILE=tile)
-    r = subprocess.run([sys.executable, "-c", CHILD, ROOT, tile], env=env, capture_output=True, text=True,
-                       timeout=600)
-    assert r.returncode == 0 and "ok" in r.stdout, r.stdout + r.stderr
+    _run_child(tile, "1x200x256,130x300x512,600x520x1280,1025x264x256")
+
+
+# Shapes whose tile count leaves a short last wave on a 148-SM part, so the
+# tail tiles are split along K and summed by tail_reduce_kernel:
+#   1280 x 3840: pair 256 x 256 -> 75 tiles = 74 + 1; pair 256 x 128 -> 150 =
+#                2 x 74 + 2; 128 x 256 -> 150 = 148 + 2
+#   1100 x 3900 (ragged rows and columns): pair 256 x 256 -> 80 = 74 + 6;
+#                pair 256 x 128 -> 155 = 2 x 74 + 7
+@pytest.mark.parametrize("tile", ["pair:256", "pair:128", "normal:256"])
+def test_split_last_wave_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
+    _run_child(tile, "1280x3840x1024,1100x3900x1024")

@@ -117,7 +117,7 @@ def test_per_tensor_sweep(oracle_mod, gpu, m):
     assert fq.device_status() == 0
 
 
-@pytest.mark.parametrize("m,k", [(1, 8), (3, 24), (1, 2048), (2048, 2048), (16384, 2048), (5, 7168)])
+@pytest.mark.parametrize("m,k", [(1, 8), (3, 24), (1, 2048), (2048, 2048), (16384, 2048), (5, 7168), (4096, 7168)])
 def test_per_tensor_other_shapes(oracle_mod, gpu, m, k):
     x = inputs.activations_per_tensor(m, k=k, seed=m + k)
     q_ref, s_ref = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))

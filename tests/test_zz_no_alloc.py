@@ -12,6 +12,8 @@ GEMM tolerance the other tests use, and against the allocating entry point
 fp8_block_gemm.  This file is collected last
 so a stop-at-first-failure run has already run every other test.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -71,13 +73,17 @@ def test_noalloc_cuts_the_split_tail_to_its_scratch(oracle_mod, cuda_lib, gpu):
     m, n, k = 4000, 7100, 4608
     assert lib.fp8_block_gemm_workspace_size(m, n, k) > _abi.NOALLOC_MAX_SCRATCH_BYTES
     sms = torch.cuda.get_device_properties(gpu).multi_processor_count
-    tiles_p, tiles_q = -(-m // 128), -(-n // 256)
-    tail = (tiles_p * tiles_q) % sms
-    assert 0 < tail <= sms // 2
+    plan = (ctypes.c_int * 11)()
+    ws = ctypes.c_size_t(0)
+    assert lib.fp8q_gemm_plan(m, n, k, sms, ctypes.c_size_t(-1).value, plan, ctypes.byref(ws)) == FP8Q_OK
+    pair, bn, tiles_p, tiles_q, tail = plan[1], plan[2], plan[5], plan[6], plan[9]
+    rows = 256 if pair else 128               # a CTA pair computes 256-row tiles
+    assert tiles_p == -(-m // rows) and tiles_q == -(-n // bn)
+    assert tail == (tiles_p * tiles_q) % (sms // 2 if pair else sms) and tail > 0
     in_tail = np.zeros((m, n), dtype=bool)
     for t in range(tiles_p * tiles_q - tail, tiles_p * tiles_q):
         tp, tq = t % tiles_p, t // tiles_p
-        in_tail[tp * 128:tp * 128 + 128, tq * 256:tq * 256 + 256] = True
+        in_tail[tp * rows:tp * rows + rows, tq * bn:tq * bn + bn] = True
     ms, ns = np.nonzero(in_tail)
     for seed in (303, 404):
         qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=seed)
