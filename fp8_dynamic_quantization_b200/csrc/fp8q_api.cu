@@ -218,6 +218,26 @@ int launch_status(int n = 1) {
     return FP8Q_OK;
 }
 
+// CTAs of `kernel` (kQuantThreads threads, no dynamic shared memory) that
+// fit on the device at once: the grid of the chunked streaming kernels,
+// which stride over their chunks.
+template <auto kernel>
+int64_t resident_ctas(int sms) {
+    static const int per_sm = [] {
+        int n = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kernel, kQuantThreads, 0) != cudaSuccess) n = 0;
+        cudaGetLastError();
+        return std::max(1, std::min(n, kBlocksPerSm));
+    }();
+    return int64_t(per_sm) * sms;
+}
+
+// Grid of a chunked kernel: one CTA per chunk, at most what fits at once.
+template <auto kernel>
+int chunk_grid(int64_t chunks, int sms) {
+    return int(std::max<int64_t>(1, std::min(chunks, resident_ctas<kernel>(sms))));
+}
+
 // Streaming grid: enough CTAs for the data, capped at kBlocksPerSm per SM.
 int stream_grid(int64_t nvec, int sms) {
     const int64_t need = (nvec + int64_t(kQuantThreads) * kStreamU - 1) /
@@ -550,13 +570,36 @@ int fp8_act_quant_per_tensor(const void* x, int64_t M, int64_t K, int64_t ldx, u
         if (e != cudaSuccess) { cudaGetLastError(); return FP8Q_ERR_CUDA; }
         return launch_status(1);
     }
-    const int grid = stream_grid(nvec, d->sms);
     uint32_t* partials = ws;
+    const uint16_t* xs = static_cast<const uint16_t*>(x);
+    const bool keep = keep_in_l2(d, M * ldx * 2);
+    if (contig) {
+        constexpr int64_t kChunk = int64_t(kQuantThreads) * kStreamU;
+        const int64_t chunks = (nvec + kChunk - 1) / kChunk;
+        const uint4* xv = static_cast<const uint4*>(x);
+        uint2* qv = reinterpret_cast<uint2*>(q);
+        const int ga = keep ? chunk_grid<amax_contig_kernel<kStreamU, true>>(chunks, d->sms)
+                            : chunk_grid<amax_contig_kernel<kStreamU, false>>(chunks, d->sms);
+        const int gp = keep ? chunk_grid<apply_contig_kernel<kStreamU, false, true>>(chunks, d->sms)
+                            : chunk_grid<apply_contig_kernel<kStreamU, false, false>>(chunks, d->sms);
+        if (log_enabled())
+            std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: amax grid=%d, apply grid=%d, %lld chunks%s\n",
+                         (long long)M, (long long)K, ga, gp, (long long)chunks, keep ? ", kept in L2" : "");
+        if (keep) {
+            launch(amax_contig_kernel<kStreamU, true>, dim3(ga), dim3(kQuantThreads), 0, st, 1u, xv, nvec, partials);
+            launch(apply_contig_kernel<kStreamU, false, true>, dim3(gp), dim3(kQuantThreads), 0, st, 1u, xv, nvec,
+                   (const uint32_t*)partials, ga, qv, scale);
+        } else {
+            launch(amax_contig_kernel<kStreamU, false>, dim3(ga), dim3(kQuantThreads), 0, st, 1u, xv, nvec, partials);
+            launch(apply_contig_kernel<kStreamU, false, false>, dim3(gp), dim3(kQuantThreads), 0, st, 1u, xv, nvec,
+                   (const uint32_t*)partials, ga, qv, scale);
+        }
+        return launch_status(2);
+    }
+    const int grid = stream_grid(nvec, d->sms);
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] per_tensor M=%lld K=%lld: amax+apply grid=%d\n",
                      (long long)M, (long long)K, grid);
-    const uint16_t* xs = static_cast<const uint16_t*>(x);
-    const bool keep = keep_in_l2(d, M * ldx * 2);
     if (contig && keep) {
         launch(amax_partial_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
                partials);
@@ -598,10 +641,21 @@ int fp8_act_amax(const void* x, int64_t M, int64_t K, int64_t ldx, uint32_t* ama
     if (M == 0 || K == 0)
         return cudaMemsetAsync(amax_bits, 0, 4, st) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
     const int64_t vpr = K / 8, nvec = M * vpr;
-    const int grid = stream_grid(nvec, d->sms);
     uint32_t* partials = static_cast<uint32_t*>(workspace);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     const bool keep = keep_in_l2(d, M * ldx * 2);      // for an apply call that follows
+    if (ldx == K) {
+        constexpr int64_t kChunk = int64_t(kQuantThreads) * kStreamU;
+        const int64_t chunks = (nvec + kChunk - 1) / kChunk;
+        const uint4* xv = static_cast<const uint4*>(x);
+        const int ga = keep ? chunk_grid<amax_contig_kernel<kStreamU, true>>(chunks, d->sms)
+                            : chunk_grid<amax_contig_kernel<kStreamU, false>>(chunks, d->sms);
+        if (keep) launch(amax_contig_kernel<kStreamU, true>, dim3(ga), dim3(kQuantThreads), 0, st, 1u, xv, nvec, partials);
+        else launch(amax_contig_kernel<kStreamU, false>, dim3(ga), dim3(kQuantThreads), 0, st, 1u, xv, nvec, partials);
+        launch(reduce_partials_kernel, dim3(1), dim3(kQuantThreads), 0, st, 1u, (const uint32_t*)partials, ga, amax_bits);
+        return launch_status(2);
+    }
+    const int grid = stream_grid(nvec, d->sms);
     if (ldx == K && keep)
         launch(amax_partial_kernel<kStreamU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
                partials);
@@ -632,9 +686,24 @@ int fp8_act_quant_apply(const void* x, int64_t M, int64_t K, int64_t ldx,
         if (scale) launch(scale_only_kernel, dim3(1), dim3(32), 0, st, 1u, amax_bits, scale);
         return launch_status();
     }
-    const int grid = stream_grid(nvec, d->sms);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
     const bool keep = keep_in_l2(d, M * ldx * 2);      // an amax call before this one kept x in L2
+    if (ldx == K && ldq == K) {
+        constexpr int64_t kChunk = int64_t(kQuantThreads) * kStreamU;
+        const int64_t chunks = (nvec + kChunk - 1) / kChunk;
+        const uint4* xv = static_cast<const uint4*>(x);
+        uint2* qv = reinterpret_cast<uint2*>(q);
+        if (keep)
+            launch(apply_contig_kernel<kStreamU, true, true>,
+                   dim3(chunk_grid<apply_contig_kernel<kStreamU, true, true>>(chunks, d->sms)), dim3(kQuantThreads), 0,
+                   st, 1u, xv, nvec, amax_bits, 1, qv, scale);
+        else
+            launch(apply_contig_kernel<kStreamU, true, false>,
+                   dim3(chunk_grid<apply_contig_kernel<kStreamU, true, false>>(chunks, d->sms)), dim3(kQuantThreads), 0,
+                   st, 1u, xv, nvec, amax_bits, 1, qv, scale);
+        return launch_status();
+    }
+    const int grid = stream_grid(nvec, d->sms);
     if (ldx == K && ldq == K && keep)
         launch(apply_kernel<kStreamU, true, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, nvec, vpr, ldx,
                amax_bits, 1, q, ldq, scale);
@@ -664,6 +733,21 @@ static int run_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int64_t G = K / 128, groups = M * G;
     constexpr int kGroupU = 2;        // groups per thread per iteration (8 threads a group)
+    const bool contig = ldx == K && ldq == K;
+    if (contig) {
+        constexpr int64_t kChunk = int64_t(kQuantThreads / 8) * kGroupU;
+        const int64_t chunks = (groups + kChunk - 1) / kChunk;
+        const uint4* xv = static_cast<const uint4*>(x);
+        uint2* qv = reinterpret_cast<uint2*>(q);
+        const int grid = e8 ? chunk_grid<group128_contig_kernel<kGroupU, true>>(chunks, d->sms)
+                            : chunk_grid<group128_contig_kernel<kGroupU, false>>(chunks, d->sms);
+        if (log_enabled())
+            std::fprintf(stderr, "[fp8q] group128%s M=%lld K=%lld: grid=%d, %lld chunks\n", e8 ? " ue8m0" : "",
+                         (long long)M, (long long)K, grid, (long long)chunks);
+        if (e8) launch(group128_contig_kernel<kGroupU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xv, qv, scales, groups);
+        else launch(group128_contig_kernel<kGroupU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xv, qv, scales, groups);
+        return launch_status();
+    }
     const int64_t need = (groups * 8 + int64_t(kQuantThreads) * kGroupU - 1) /
                          (int64_t(kQuantThreads) * kGroupU);
     const int grid = int(std::max<int64_t>(1, std::min<int64_t>(need, int64_t(d->sms) * kBlocksPerSm)));
@@ -671,13 +755,8 @@ static int run_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
         std::fprintf(stderr, "[fp8q] group128%s M=%lld K=%lld: grid=%d\n", e8 ? " ue8m0" : "",
                      (long long)M, (long long)K, grid);
     const uint16_t* xs = static_cast<const uint16_t*>(x);
-    const bool contig = ldx == K && ldq == K;
-    if (e8 && contig)
-        launch(group128_quant_kernel<kGroupU, true, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
-    else if (e8)
+    if (e8)
         launch(group128_quant_kernel<kGroupU, false, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
-    else if (contig)
-        launch(group128_quant_kernel<kGroupU, true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     else
         launch(group128_quant_kernel<kGroupU, false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xs, ldx, q, ldq, scales, groups, G);
     return launch_status();

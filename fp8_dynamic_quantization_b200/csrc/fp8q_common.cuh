@@ -17,7 +17,8 @@
 //
 // RN(x / scale) without a division per element: with r = RN(1/scale)
 // (__frcp_rn, once per scale), q0 = RN(x*r), rem = x - q0*scale (one fma),
-// q = fma(rem, r, q0) -- Markstein's correction step (P. Markstein,
+// q = fma(rem, r, q0), two values per f32x2 instruction (quant8_x2), the
+// sign of each code then taken from x -- Markstein's correction step (P. Markstein,
 // "Computation of elementary functions on the IBM RISC System/6000
 // processor", IBM J. Res. Dev. 34(1), 1990).  Here x is a bf16 value and
 // scale = RN(amax/448) with amax a bf16 value, so only 128 x 128 pairs of
@@ -82,11 +83,29 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Packed fp32 pairs: two fp32 values in one 64-bit register, for the
+// sm_100 f32x2 arithmetic (one instruction for both lanes of the pair).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ void f32x2_split(uint64_t v, float& lo, float& hi) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma_f32x2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // A scale and what dividing by it needs.
 struct Scale {
     float s;      // the scale
     float r;      // RN(1/s)
     int mode;     // 0: s == 0; 1: reciprocal-corrected division; 2: IEEE division
+    uint64_t r2;  // (r, r) packed
+    uint64_t ns2; // (-s, -s) packed
 };
 
 __device__ __forceinline__ Scale make_scale(float s) {
@@ -94,17 +113,9 @@ __device__ __forceinline__ Scale make_scale(float s) {
     d.s = s;
     d.r = __frcp_rn(s);
     d.mode = (s == 0.0f) ? 0 : (s >= 0x1p-90f && s <= 0x1p126f) ? 1 : 2;
+    d.r2 = f32x2(d.r, d.r);
+    d.ns2 = f32x2(-s, -s);
     return d;
-}
-
-// RN(x / s) for finite |x| <= amax and 2^-90 <= s <= 2^126 (see above).
-// The remainder is formed negated, q0*s - x, so that x = -0 yields -0
-// ((-0) + (+0) would round to +0 in the other order); for every nonzero
-// quotient the result is the same, round-to-nearest being sign-symmetric.
-__device__ __forceinline__ float div_fast(float x, const Scale& d) {
-    const float q0 = __fmul_rn(x, d.r);
-    const float nrem = __fmaf_rn(q0, d.s, -x);
-    return __fmaf_rn(-nrem, d.r, q0);
 }
 
 // Signed-zero codes of one bf16 pair (the zero-scale convention).
@@ -113,15 +124,33 @@ __device__ __forceinline__ uint32_t zero_pair(uint32_t w) {
 }
 
 // Codes of 8 bf16 values for a scale in the reciprocal-corrected range
-// (Scale::mode == 1) and values no larger than the amax.
-__device__ __forceinline__ uint2 quant8_fast(const uint4& v, const Scale& d) {
+// (Scale::mode == 1) and values no larger than the amax, two values per
+// instruction: q0 = RN(x*r) (an fma with -0 added, which is the product
+// itself, signed zeros included), rem = RN(x - q0*s) (exact), q =
+// RN(q0 + rem*r).  This is the step above with the remainder's sign
+// flipped, which gives the same quotient for every x except x = -0, where
+// it gives +0; so the sign bit of every code is then set from x itself (the
+// sign of x / s is the sign of x for every x, zeros and underflows
+// included).  Checked on the CPU for every bf16 x with |x| <= amax against
+// RN(x / s) for every finite bf16 amax with s in the range above
+// (1,031,103,648 pairs, codes equal), and on the GPU by the exhaustive
+// (x, amax) test.
+__device__ __forceinline__ uint2 quant8_x2(const uint4& v, uint64_t r2, uint64_t ns2) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const uint64_t nz2 = f32x2(-0.0f, -0.0f);
     uint32_t c[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(div_fast(bf16_lo(w[i]), d), div_fast(bf16_hi(w[i]), d));
+    for (int i = 0; i < 4; ++i) {
+        const uint64_t x2 = f32x2(bf16_lo(w[i]), bf16_hi(w[i]));
+        const uint64_t q0 = fma_f32x2(x2, r2, nz2);
+        const uint64_t rem = fma_f32x2(q0, ns2, x2);
+        float lo, hi;
+        f32x2_split(fma_f32x2(rem, r2, q0), lo, hi);
+        c[i] = cvt_e4m3x2(lo, hi);
+    }
     uint2 r;
-    r.x = c[0] | (c[1] << 16);
-    r.y = c[2] | (c[3] << 16);
+    r.x = (c[0] | (c[1] << 16)) | (__byte_perm(v.x, v.y, 0x7531) & 0x80808080u);
+    r.y = (c[2] | (c[3] << 16)) | (__byte_perm(v.z, v.w, 0x7531) & 0x80808080u);
     return r;
 }
 
@@ -135,8 +164,7 @@ __device__ __forceinline__ uint2 quant8(const uint4& v, const Scale& d, bool exa
 #pragma unroll
         for (int i = 0; i < 4; ++i) c[i] = zero_pair(w[i]);
     } else if (d.mode == 1 && !exact) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(div_fast(bf16_lo(w[i]), d), div_fast(bf16_hi(w[i]), d));
+        return quant8_x2(v, d.r2, d.ns2);
     } else {
 #pragma unroll
         for (int i = 0; i < 4; ++i)

@@ -184,6 +184,146 @@ apply_kernel(const uint16_t* __restrict__ x, int64_t nvec, int64_t vec_per_row, 
 }
 
 // ---------------------------------------------------------------------------
+// Contiguous tensors (row stride == row length): the same passes over
+// chunks of kQuantThreads x U consecutive 16-byte vectors.  Thread t of a
+// CTA handles vectors t, t + 256, ... of its chunk, so every load and store
+// of the chunk is one base pointer plus a constant offset, and only the
+// last, partial chunk checks bounds; the grid strides over chunks.  This
+// keeps the index arithmetic out of the per-vector work, which (with the
+// per-element division) is what bounds these kernels when x is in L2.
+// ---------------------------------------------------------------------------
+template <int U, bool KEEP = false>
+__global__ void __launch_bounds__(kQuantThreads)
+amax_contig_kernel(const uint4* __restrict__ x, int64_t nvec, uint32_t* __restrict__ partials) {
+    pdl_begin();
+    __shared__ uint32_t red[kQuantThreads / 32];
+    constexpr int kChunk = kQuantThreads * U;
+    const uint64_t pol = KEEP ? l2_policy_evict_last() : 0ull;
+    const int64_t nchunks = (nvec + kChunk - 1) / kChunk;
+    uint32_t m = 0;
+    for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        const int64_t base = c * kChunk + threadIdx.x;
+        const uint4* xp = x + base;
+        uint4 v[U];
+        if (c * kChunk + kChunk <= nvec) {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                v[u] = KEEP ? ld_stream16_hint(xp + u * kQuantThreads, pol) : ld_stream16(xp + u * kQuantThreads);
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                v[u] = base + u * kQuantThreads < nvec ? ld_stream16(xp + u * kQuantThreads) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) m = max(m, absmax8(v[u]));
+    }
+    m = block_max<kQuantThreads>(m, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = m;
+}
+
+// Apply pass over chunks, last chunk first (the amax pass read the end of
+// the tensor last, so that part is the likeliest to be in L2).  CHECK and
+// KEEP as in apply_kernel.
+template <int U, bool CHECK, bool KEEP = false>
+__global__ void __launch_bounds__(kQuantThreads)
+apply_contig_kernel(const uint4* __restrict__ x, int64_t nvec, const uint32_t* __restrict__ partials,
+                    int nparts, uint2* __restrict__ q, float* __restrict__ scale_out) {
+    pdl_begin();
+    __shared__ uint32_t red[kQuantThreads / 32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < nparts; i += kQuantThreads)
+        m = max(m, __ldcg(partials + i) & 0x7FFFu);
+    m = block_max<kQuantThreads>(m, red);
+    const Scale d = make_scale(scale_from_amax_bits(m));
+    if (blockIdx.x == 0 && threadIdx.x == 0 && scale_out) *scale_out = d.s;
+
+    constexpr int kChunk = kQuantThreads * U;
+    const uint64_t pol = KEEP ? l2_policy_evict_first() : 0ull;
+    const int64_t nchunks = (nvec + kChunk - 1) / kChunk;
+    const bool fast = d.mode == 1 && !CHECK;
+    for (int64_t c = nchunks - 1 - blockIdx.x; c >= 0; c -= gridDim.x) {
+        const int64_t base = c * kChunk + threadIdx.x;
+        const uint4* xp = x + base;
+        uint2* qp = q + base;
+        if (c * kChunk + kChunk <= nvec) {
+            uint4 v[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u)
+                v[u] = KEEP ? ld_stream16_hint(xp + u * kQuantThreads, pol) : ld_stream16(xp + u * kQuantThreads);
+            if (fast) {
+#pragma unroll
+                for (int u = 0; u < U; ++u) st_stream8(qp + u * kQuantThreads, quant8_x2(v[u], d.r2, d.ns2));
+            } else {
+#pragma unroll
+                for (int u = 0; u < U; ++u)
+                    st_stream8(qp + u * kQuantThreads, quant8(v[u], d, CHECK && absmax8(v[u]) > m));
+            }
+        } else {
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                if (base + u * kQuantThreads < nvec) {
+                    const uint4 v = ld_stream16(xp + u * kQuantThreads);
+                    st_stream8(qp + u * kQuantThreads, quant8(v, d, CHECK && absmax8(v) > m));
+                }
+            }
+        }
+    }
+}
+
+// Per-1x128-group quantisation of a contiguous [M, K] tensor: chunks of
+// U x 32 consecutive groups (8 threads per group as in
+// group128_quant_kernel; lanes 8j..8j+7 of a warp own group 4w+j of each
+// 32-group slice, so a warp's four groups are in or out of range together
+// except in the last chunk).
+template <int U, bool E8 = false>
+__global__ void __launch_bounds__(kQuantThreads)
+group128_contig_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void* __restrict__ scales,
+                       int64_t groups) {
+    pdl_begin();
+    constexpr int kSlice = kQuantThreads / 8;               // groups per slice (32)
+    constexpr int kChunk = kSlice * U;                      // groups per chunk
+    const int sub = threadIdx.x & 7;
+    const int gl = threadIdx.x >> 3;                        // group within a slice
+    const int64_t nchunks = (groups + kChunk - 1) / kChunk;
+    for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        const int64_t g0 = c * kChunk + gl;                 // this thread's group in slice 0
+        const uint4* xp = x + g0 * 16 + sub;                // a group is 16 vectors
+        uint2* qp = q + g0 * 16 + sub;
+        const bool full = c * kChunk + kChunk <= groups;
+        uint4 a[U], b[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const bool ok = full || g0 + u * kSlice < groups;
+            a[u] = ok ? ld_stream16(xp + u * kSlice * 16) : make_uint4(0, 0, 0, 0);
+            b[u] = ok ? ld_stream16(xp + u * kSlice * 16 + 8) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t g = g0 + u * kSlice;
+            // a warp's four groups: test the first, so the shuffles stay warp-uniform
+            if (!full && ((g - (gl & 3)) >= groups)) break;
+            uint32_t m = max(absmax8(a[u]), absmax8(b[u]));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 4));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+            m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+            if (!full && g >= groups) continue;
+            if (E8) {
+                const uint32_t sb = e8m0_from_amax_bits(m);
+                const float inv = e8m0_inverse(sb);
+                st_stream8(qp + u * kSlice * 16, quant8_pow2(a[u], inv));
+                st_stream8(qp + u * kSlice * 16 + 8, quant8_pow2(b[u], inv));
+                if (sub == 0) static_cast<uint8_t*>(scales)[g] = uint8_t(sb);
+            } else {
+                const Scale d = make_scale(scale_from_amax_bits(m));
+                st_stream8(qp + u * kSlice * 16, quant8(a[u], d));
+                st_stream8(qp + u * kSlice * 16 + 8, quant8(b[u], d));
+                if (sub == 0) static_cast<float*>(scales)[g] = d.s;
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // Per-tensor, single launch, for tensors that fit in the registers of one
 // thread-block cluster (up to 8 CTAs of NT threads, U vectors per thread;
 // a single CTA is launched without a cluster and needs no exchange).  Each CTA reduces its values to one partial max in shared
