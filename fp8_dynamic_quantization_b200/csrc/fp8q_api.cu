@@ -233,6 +233,8 @@ int64_t resident_ctas(int sms) {
 }
 
 // Grid of a chunked kernel: one CTA per chunk, at most what fits at once.
+// (A grid that gives every CTA the same number of chunks measured slower
+// back to back: 21.6 against 20.0 us per-tensor at 4096 x 7168.)
 template <auto kernel>
 int chunk_grid(int64_t chunks, int sms) {
     return int(std::max<int64_t>(1, std::min(chunks, resident_ctas<kernel>(sms))));
