@@ -69,7 +69,9 @@ def _run_child(tile, shapes):
 @pytest.mark.parametrize("tile", ["normal:128", "normal:192", "normal:256", "pair:256", "pair:128",
                                   "swap:16", "swap:32", "swap:64", "swap:128:3"])
 def test_gemm_mode_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
-    _run_child(tile, "1x200x256,130x300x512,600x520x1280,1025x264x256")
+    # 257 x 384 x 640: five K blocks, so the last two-K-block round of a CTA
+    # pair's 256 x 128 tiles holds one
+    _run_child(tile, "1x200x256,130x300x512,600x520x1280,1025x264x256,257x384x640")
 
 
 # Shapes whose tile count leaves a short last wave on a 148-SM part, so the
@@ -78,6 +80,7 @@ def test_gemm_mode_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
 #                2 x 74 + 2; 128 x 256 -> 150 = 148 + 2
 #   1100 x 3900 (ragged rows and columns): pair 256 x 256 -> 80 = 74 + 6;
 #                pair 256 x 128 -> 155 = 2 x 74 + 7
+#   1280 x 3840 x 1152: nine K blocks split into 4 ranges (2, 2, 2, 3 blocks)
 @pytest.mark.parametrize("tile", ["pair:256", "pair:128", "normal:256"])
 def test_split_last_wave_matches_oracle(gpu, cuda_lib, oracle_mod, tile):
-    _run_child(tile, "1280x3840x1024,1100x3900x1024")
+    _run_child(tile, "1280x3840x1024,1100x3900x1024,1280x3840x1152")
