@@ -946,15 +946,16 @@ tail_reduce_kernel(const float* __restrict__ ws, int tail_tiles, int splits, int
         if (m >= M || n >= N) continue;
         const float* src = ws + (int64_t(tt) * splits * tile_rows + r) * bn + c;
         float a[4] = {0.f, 0.f, 0.f, 0.f};
-        // loads issued 6 at a time, added in split order
-        for (int s0 = 0; s0 < splits; s0 += 6) {
-            float4 v[6];
+        // loads issued 18 at a time (all of them for the usual split
+        // counts), added in split order
+        for (int s0 = 0; s0 < splits; s0 += 18) {
+            float4 v[18];
 #pragma unroll
-            for (int t = 0; t < 6; ++t)
+            for (int t = 0; t < 18; ++t)
                 v[t] = s0 + t < splits ? __ldcs(reinterpret_cast<const float4*>(src + int64_t(s0 + t) * slot))
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-            for (int t = 0; t < 6; ++t)
+            for (int t = 0; t < 18; ++t)
                 if (s0 + t < splits) { a[0] += v[t].x; a[1] += v[t].y; a[2] += v[t].z; a[3] += v[t].w; }
         }
         if (n + 4 <= N) {

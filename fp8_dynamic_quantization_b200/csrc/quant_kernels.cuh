@@ -6,12 +6,15 @@
 // dynamic-quant amax grid to the input", Description: a fixed 1024-block
 // grid with a 1024-way atomic sets a data-independent floor).
 //
-//  group128_quant_kernel     one pass: amax of each 1x128 group, its scale,
-//                            codes ("How to Profile DeepSeek-V3 Inference
+//  group128_contig_kernel /  one pass: amax of each 1x128 group, its scale,
+//  group128_quant_kernel     codes ("How to Profile DeepSeek-V3 Inference
 //                            Kernels Using Triton Autotuning", Benchmarking
-//                            the Activation Quantization Kernel).
-//  amax_partial_kernel       per-tensor amax, one partial max per CTA.
-//  apply_kernel              per-tensor apply pass: reduces the partials
+//                            the Activation Quantization Kernel); the first
+//                            for contiguous tensors, the second for strided.
+//  amax_contig_kernel /      per-tensor amax, one partial max per CTA
+//  amax_partial_kernel       (contiguous / strided).
+//  apply_contig_kernel /     per-tensor apply pass (contiguous / strided):
+//  apply_kernel              reduces the partials
 //                            (or reads one amax word), computes the scale,
 //                            writes codes.  Walks the tensor backwards, so
 //                            the part of x the amax pass read last is still

@@ -7,6 +7,8 @@ prefill shapes (the launch configurations the benchmark times) at sampled
 points -- every corner and tail tile, whole rows and columns, and random
 points -- which the oracle evaluates one by one.
 """
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -107,18 +109,19 @@ def test_gemm_prefill_shapes(oracle_mod, gpu, n):
 
 
 def tail_region(M, N, K, sms):
-    """Rows and columns of the tiles the planner splits along K (128 x 256
-    tiles past the last full wave of `sms` CTAs, when that last wave fills at
-    most half the SMs); empty when no tile is split."""
-    tiles_p, tiles_q = -(-M // 128), -(-N // 256)
+    """Rows and columns of the tiles the launch plan splits along K (the
+    tiles past the last full wave, when that wave fills at most half the
+    SMs, or half the CTA pairs); empty when no tile is split."""
+    plan = (ctypes.c_int * 11)()
+    ws = ctypes.c_size_t(0)
+    assert fq.library().fp8q_gemm_plan(M, N, K, sms, ctypes.c_size_t(-1).value, plan, ctypes.byref(ws)) == 0
+    pair, bn, tiles_p, tiles_q, tail = plan[1], plan[2], plan[5], plan[6], plan[9]
+    rows = 256 if pair else 128                 # a CTA pair computes 256-row tiles
     tiles = tiles_p * tiles_q
-    tail = tiles % sms
-    if M <= 512 or tiles <= sms or tail == 0 or min(sms // tail, (K // 128) // 2) < 2:
-        return []
     out = []
     for t in range(tiles - tail, tiles):
         tp, tq = t % tiles_p, t // tiles_p
-        out.append((np.arange(tp * 128, min(M, tp * 128 + 128)), np.arange(tq * 256, min(N, tq * 256 + 256))))
+        out.append((np.arange(tp * rows, min(M, tp * rows + rows)), np.arange(tq * bn, min(N, tq * bn + bn))))
     return out
 
 
