@@ -142,7 +142,7 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4>();
                 if (e == cudaSuccess) e = set_gemm_smem<256, false, 4, false, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, false, true>();
-                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 5, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, true>();
@@ -355,7 +355,7 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
     pl.pair = row->mode == kPair && !no_pair;
     pl.bn = row->bn;
     pl.stages = pl.swap ? (pl.bn == 16 ? 12 : pl.bn == 32 ? 10 : pl.bn == 64 ? 8 : 6)
-                        : pl.pair ? (pl.bn == 256 ? 6 : 8) : (pl.bn == 192 ? 5 : pl.bn == 256 ? 4 : 6);
+                        : pl.pair ? (pl.bn == 256 ? 5 : 8) : (pl.bn == 192 ? 5 : pl.bn == 256 ? 4 : 6);
     const int G = int(K / 128);
     const int64_t rows_p = pl.swap ? N : M, rows_q = pl.swap ? M : N;
     const int tile_rows = pl.pair ? 256 : 128;
@@ -403,6 +403,11 @@ GemmPlan plan_gemm(int64_t M, int64_t N, int64_t K, int sms, bool no_pair = fals
     return pl;
 }
 
+// Map of the bf16 output Y [M, N] (row pitch ldy elements, 16-byte aligned
+// base and pitch): boxes of 64 columns (128 bytes) x 32 rows, 128-byte
+// swizzle, for bulk stores of the CTA-pair tiles' epilogue.
+bool make_y_tmap(CUtensorMap* m, const void* base, int64_t M, int64_t N, int64_t ldy);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -436,6 +441,18 @@ bool make_tmap(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int64_
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool make_y_tmap(CUtensorMap* m, const void* base, int64_t M, int64_t N, int64_t ldy) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cuuint64_t(N), cuuint64_t(M)};
+    cuuint64_t strides[1] = {cuuint64_t(ldy) * 2};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Map of an fp32 scale matrix [rows, G] (row pitch G floats, G % 4 == 0,
 // 16-byte aligned base): boxes of 4 consecutive K-block scales x box_rows
 // rows, no swizzle; rows past the end read as zero.
@@ -454,10 +471,10 @@ bool make_scale_tmap(CUtensorMap* m, const float* base, int64_t rows, int64_t G,
 // tsa/tsb: scale maps (staged-scale variants only; the others ignore them)
 template <int BN, bool SWAP, int STAGES, bool PAIR = false, int SM = 0, bool SS = false>
 void launch_gemm(const CUtensorMap& tp, const CUtensorMap& tq, const CUtensorMap& tsa, const CUtensorMap& tsb,
-                 const GemmParams& p, int grid, cudaStream_t st) {
+                 const GemmParams& p, int grid, cudaStream_t st, const CUtensorMap* ty = nullptr) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
     launch(block_gemm_kernel<BN, SWAP, STAGES, PAIR, SM, SS>, dim3(unsigned(grid)), dim3(C::kThreads),
-           C::kSmemBytes, st, PAIR ? 2u : 1u, tp, tq, tsa, tsb, p);
+           C::kSmemBytes, st, PAIR ? 2u : 1u, tp, tq, tsa, tsb, ty ? *ty : tp, p);
 }
 
 // ------------------------------------------------------------------ no-alloc GEMM scratch
@@ -911,6 +928,14 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return FP8Q_ERR_CUDA;
     p.wait_budget = wait_budget_cycles();
     p.status_slot = uint8_t(status_slot(d->index, st));
+    // CTA-pair 256 x 256 tiles with fp32 block scales store Y in bulk from
+    // shared memory when Y's base and row pitch are 16-byte aligned.
+    CUtensorMap ty = tp;
+    p.ystore = 0;
+    if (pl.pair && pl.bn == 256 && mode == 0 && aligned16(y) && (ldy * 2) % 16 == 0) {
+        if (!make_y_tmap(&ty, y, M, N, ldy)) return FP8Q_ERR_CUDA;
+        p.ystore = 1;
+    }
     if (log_enabled())
         std::fprintf(stderr, "[fp8q] gemm M=%lld N=%lld K=%lld: %s%s bn=%d stages=%d splits=%d units=%d grid=%d"
                              " tail=%dx%d\n",
@@ -976,7 +1001,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
             default: launch_gemm<128, true, 6>(tp, tq, tsa, tsb, p, pl.grid, st); break;
         }
     } else if (pl.pair) {
-        if (pl.bn == 256) launch_gemm<256, false, 6, true>(tp, tq, tsa, tsb, p, pl.grid, st);
+        if (pl.bn == 256) launch_gemm<256, false, 5, true>(tp, tq, tsa, tsb, p, pl.grid, st, &ty);
         else launch_gemm<128, false, 8, true>(tp, tq, tsa, tsb, p, pl.grid, st);
     } else {
         if (pl.bn == 192) launch_gemm<192, false, 5>(tp, tq, tsa, tsb, p, pl.grid, st);

@@ -101,6 +101,7 @@ struct GemmParams {
     uint8_t sf_words;    // ue8m0: 4 scale bytes readable as one word (G % 4 == 0, 4-byte aligned)
     uint8_t pdl;         // the weights do not depend on the previous kernel (it produces A and sa)
     uint8_t status_slot; // error word of the launching stream (g_stream_status index)
+    uint8_t ystore;      // TS tiles: Y has a tensor map (tmY) for bulk stores from shared memory
     long long wait_budget;  // SM clock cycles a barrier wait may take before giving up
 };
 static_assert(sizeof(GemmParams) <= 104, "GemmParams size");
@@ -125,6 +126,12 @@ struct GemmCfg {
                   "register split exceeds the launch allocation");
     static_assert(kEpiWG <= 3, "at most three promotion warpgroups");
     static constexpr int kTileRows = PAIR ? 256 : 128;         // rows of P per work unit
+    // TS: the epilogue of whole tiles converts Y to bf16 into a shared-memory
+    // tile (each promotion warp its 32 rows x kCW columns, 128-byte
+    // swizzled) and bulk-stores it, so the promotion warps go back to the
+    // next tile's partials without waiting for the global stores.
+    static constexpr bool TS = PAIR && BN == 256 && SM == 0;
+    static constexpr int kYBytes = TS ? 128 * BN * 2 : 0;
     static constexpr int kPBytes = 128 * 128;                  // 128 rows x 128 K bytes
     static constexpr int kQRows = PAIR ? BN / 2 : BN;         // B (or A) rows this CTA loads
     static constexpr int kQBytes = kQRows * 128;
@@ -148,7 +155,7 @@ struct GemmCfg {
     static constexpr int kSbRows = BN / 128;                   // column blocks per tile (SS)
     static constexpr int kScaleSlotBytes = 2048 + 128;         // 128 x 4 fp32, then kSbRows x 4 fp32
     static constexpr uint32_t kScaleTx = 2048 + 16 * kSbRows;  // bytes one slot receives
-    static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes
+    static constexpr size_t kSmemBytes = 1024 + size_t(STAGES) * kStageBytes + size_t(kYBytes)
                                          + size_t(kSlabFloats) * 4 + size_t(kScaleSlots) * kScaleSlotBytes
                                          + size_t(kSfSlots) * kSfSlotBytes + 512;
     static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "BN");
@@ -302,6 +309,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
                   const __grid_constant__ CUtensorMap tmQ,
                   const __grid_constant__ CUtensorMap tmSA,    // row scales [M, G] fp32 (SS only)
                   const __grid_constant__ CUtensorMap tmSB,    // column-block scales [NB, G] fp32 (SS only)
+                  const __grid_constant__ CUtensorMap tmY,     // bf16 Y [M, N], 64 x 32 boxes (TS with p.ystore)
                   const GemmParams p) {
     using C = GemmCfg<BN, SWAP, STAGES, PAIR, SM, SS>;
     constexpr bool PT = C::PT, MX = C::MX, PC = C::PC;
@@ -321,8 +329,9 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* tiles = smem;                                        // STAGES x (P | Q)
-    float* slab = reinterpret_cast<float*>(smem + size_t(STAGES) * C::kStageBytes);
-    uint8_t* sring = smem + size_t(STAGES) * C::kStageBytes + size_t(C::kSlabFloats) * 4;   // SS slots
+    uint8_t* ytile = smem + size_t(STAGES) * C::kStageBytes;      // TS: bf16 Y tile, 8 KB per promotion warp
+    float* slab = reinterpret_cast<float*>(ytile + C::kYBytes);
+    uint8_t* sring = ytile + C::kYBytes + size_t(C::kSlabFloats) * 4;   // SS slots
     uint8_t* sfring = sring + size_t(C::kScaleSlots) * C::kScaleSlotBytes;   // MX scale-factor slots
     uint64_t* bars = reinterpret_cast<uint64_t*>(sfring + size_t(C::kSfSlots) * C::kSfSlotBytes);
     uint64_t* full = bars;                        // [STAGES] TMA landed
@@ -738,7 +747,38 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
 #pragma unroll
                 for (int j = 0; j < C::kCW; ++j) acc[j] *= slab[chalf * C::kCW + j];
             }
-            if (p.splits == 1 && u < p.full_units && !SWAP && C::kCW % 64 == 0) {
+            if (C::TS && p.ystore && p.splits == 1 && u < p.full_units) {
+                // bf16 Y through shared memory: this warp's 32 rows x 128
+                // columns as two 64-column boxes (32 rows of 128 bytes, 16-byte
+                // chunk c of row r at chunk c ^ (r % 8)), then two bulk stores
+                uint8_t* wreg = ytile + size_t(e) * 8192;
+                if (lane == 0) ptx::bulk_wait_read_all();      // the previous tile's stores have read it
+                __syncwarp();
+#pragma unroll
+                for (int b = 0; b < 2; ++b) {
+#pragma unroll
+                    for (int cc = 0; cc < 8; ++cc) {
+                        const int j = b * 64 + cc * 8;
+                        uint4 w;
+                        w.x = ptx::pack_bf16x2(acc[j + 0], acc[j + 1]);
+                        w.y = ptx::pack_bf16x2(acc[j + 2], acc[j + 3]);
+                        w.z = ptx::pack_bf16x2(acc[j + 4], acc[j + 5]);
+                        w.w = ptx::pack_bf16x2(acc[j + 6], acc[j + 7]);
+                        *reinterpret_cast<uint4*>(wreg + b * 4096 + lane * 128 + ((cc ^ (lane & 7)) * 16)) = w;
+                    }
+                }
+                ptx::fence_proxy_async_shared();
+                __syncwarp();
+                if (lane == 0) {
+                    const int y0 = tp * C::kTileRows + int(rank) * 128 + quarter * 32;
+                    const int x0 = q0 + chalf * C::kCW;
+                    if (y0 < p.M) {
+                        if (x0 < p.N) ptx::tma_store_2d(&tmY, ptx::smem_u32(wreg), x0, y0);
+                        if (x0 + 64 < p.N) ptx::tma_store_2d(&tmY, ptx::smem_u32(wreg + 4096), x0 + 64, y0);
+                    }
+                    ptx::bulk_commit_group();
+                }
+            } else if (p.splits == 1 && u < p.full_units && !SWAP && C::kCW % 64 == 0) {
                 // bf16 Y, 64 columns (8 chunks) per block, stored through
                 // transpose8x8.  Writing a tile row by row took ~8000 clocks
                 // per tile with the MMA stalled behind it; this takes ~3200.
@@ -880,6 +920,7 @@ block_gemm_kernel(const __grid_constant__ CUtensorMap tmP,
         }
     }
 
+    if (C::TS && warp >= 4 && lane == 0) ptx::bulk_wait_all();   // this warp's Y stores have completed
     __syncwarp();
     ptx::tc_fence_before();
     if (PAIR) ptx::cluster_sync();      // both CTAs done with TMEM and with each other's barriers
