@@ -929,10 +929,11 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
     p.wait_budget = wait_budget_cycles();
     p.status_slot = uint8_t(status_slot(d->index, st));
     // CTA-pair 256 x 256 tiles with fp32 block scales store Y in bulk from
-    // shared memory when Y's base and row pitch are 16-byte aligned.
+    // shared memory (check_gemm_args has made Y's base and row pitch 16-byte
+    // aligned, as the tensor map needs).
     CUtensorMap ty = tp;
     p.ystore = 0;
-    if (pl.pair && pl.bn == 256 && mode == 0 && aligned16(y) && (ldy * 2) % 16 == 0) {
+    if (pl.pair && pl.bn == 256 && mode == 0) {
         if (!make_y_tmap(&ty, y, M, N, ldy)) return FP8Q_ERR_CUDA;
         p.ystore = 1;
     }
