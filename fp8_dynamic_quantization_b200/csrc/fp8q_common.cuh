@@ -54,11 +54,6 @@ __device__ __forceinline__ uint32_t absmax8(const uint4& v) {
     return max(c & 0xFFFFu, c >> 16);
 }
 
-// fp32 value of a bf16 magnitude field produced by absmax8.
-__device__ __forceinline__ float amax_bits_to_f32(uint32_t bits) {
-    return __uint_as_float(bits << 16);
-}
-
 // RN(1/448) in fp32.
 constexpr float kInvE4M3Max = 0x1.24924ap-9f;
 
