@@ -150,9 +150,9 @@ int device_info(DeviceInfo** out) {
                 if (e == cudaSuccess) e = set_gemm_smem<128, true, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 6, false, true>();
                 if (e == cudaSuccess) e = set_gemm_smem<192, false, 5, false, true>();
-                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 1>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 5, true, 1>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true, 1>();
-                if (e == cudaSuccess) e = set_gemm_smem<256, false, 6, true, 3>();
+                if (e == cudaSuccess) e = set_gemm_smem<256, false, 5, true, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<128, false, 8, true, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<16, true, 12, false, 3>();
                 if (e == cudaSuccess) e = set_gemm_smem<32, true, 10, false, 3>();
@@ -530,7 +530,7 @@ const char* fp8q_status_string(int status) {
 int fp8q_abi_version(void) { return (1 << 16) | 1; }
 
 // Host only: the launch plan fp8_block_gemm would use on a device with
-// `sms` SMs (the other scale modes run pair rows as single-CTA tiles).
+// `sms` SMs (the ue8m0 GEMM runs pair rows as single-CTA tiles).
 int fp8q_gemm_plan(int64_t M, int64_t N, int64_t K, int sms, size_t ws_cap, int* plan, size_t* ws_bytes) {
     if (M <= 0 || N <= 0 || K <= 0 || sms <= 0 || !plan || !ws_bytes) return FP8Q_ERR_INVALID_ARG;
     if (K % 128 || M > 0x7FFFFFFF || N > 0x7FFFFFFF || K > 0x7FFFFFFF) return FP8Q_ERR_UNSUPPORTED_SHAPE;
@@ -886,9 +886,10 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return cudaMemset2DAsync(y, size_t(ldy) * 2, 0, size_t(N) * 2, size_t(M), st) == cudaSuccess
                    ? FP8Q_OK : FP8Q_ERR_CUDA;
     }
-    // CTA pairs for fp32 block scales only: the one-step modes (per-tensor,
-    // per-channel) measured ~5% slower with pairs, and ue8m0 has none
-    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode != 0, ws_cap);
+    // CTA pairs for every scale mode but ue8m0, which has none (with the
+    // bulk-store epilogue the per-tensor GEMM runs 4096 x 7168 x 7168 in
+    // 168.3 against 177.2 us with pairs, the same at N = 18432-24576)
+    const GemmPlan pl = plan_gemm(M, N, K, d->sms, mode == 2, ws_cap);
     if (pl.ws_bytes > 0) {
         if (!workspace || workspace_bytes < pl.ws_bytes) return FP8Q_ERR_WORKSPACE;
         if (!aligned16(workspace)) return FP8Q_ERR_MISALIGNED;
@@ -928,12 +929,12 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         return FP8Q_ERR_CUDA;
     p.wait_budget = wait_budget_cycles();
     p.status_slot = uint8_t(status_slot(d->index, st));
-    // CTA-pair 256 x 256 tiles with fp32 block scales store Y in bulk from
-    // shared memory (check_gemm_args has made Y's base and row pitch 16-byte
-    // aligned, as the tensor map needs).
+    // CTA-pair 256 x 256 tiles store Y in bulk from shared memory
+    // (check_gemm_args has made Y's base and row pitch 16-byte aligned, as
+    // the tensor map needs).
     CUtensorMap ty = tp;
     p.ystore = 0;
-    if (pl.pair && pl.bn == 256 && mode == 0) {
+    if (pl.pair && pl.bn == 256 && mode != 2) {
         if (!make_y_tmap(&ty, y, M, N, ldy)) return FP8Q_ERR_CUDA;
         p.ystore = 1;
     }
@@ -945,7 +946,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
                      pl.stages, pl.splits, pl.units, pl.grid, pl.tail_tiles, pl.tail_splits);
     if (per_channel) {
         if (pl.pair) {
-            if (pl.bn == 256) launch_gemm<256, false, 6, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
+            if (pl.bn == 256) launch_gemm<256, false, 5, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st, &ty);
             else launch_gemm<128, false, 8, true, 3>(tp, tq, tsa, tsb, p, pl.grid, st);
         } else if (pl.swap) {
             switch (pl.bn) {
@@ -978,7 +979,7 @@ static int run_gemm(const uint8_t* qa, int64_t lda, const float* sa, const uint8
         }
     } else if (per_tensor) {
         if (pl.pair) {
-            if (pl.bn == 256) launch_gemm<256, false, 6, true, 1>(tp, tq, tsa, tsb, p, pl.grid, st);
+            if (pl.bn == 256) launch_gemm<256, false, 5, true, 1>(tp, tq, tsa, tsb, p, pl.grid, st, &ty);
             else launch_gemm<128, false, 8, true, 1>(tp, tq, tsa, tsb, p, pl.grid, st);
         } else if (pl.swap) {
             switch (pl.bn) {

@@ -130,7 +130,7 @@ struct GemmCfg {
     // tile (each promotion warp its 32 rows x kCW columns, 128-byte
     // swizzled) and bulk-stores it, so the promotion warps go back to the
     // next tile's partials without waiting for the global stores.
-    static constexpr bool TS = PAIR && BN == 256 && SM == 0;
+    static constexpr bool TS = PAIR && BN == 256 && (SM == 0 || SM == 1 || SM == 3);
     static constexpr int kYBytes = TS ? 128 * BN * 2 : 0;
     static constexpr int kPBytes = 128 * 128;                  // 128 rows x 128 K bytes
     static constexpr int kQRows = PAIR ? BN / 2 : BN;         // B (or A) rows this CTA loads

@@ -355,8 +355,8 @@ int fp8_block_gemm_noalloc(const uint8_t* qa, int64_t lda, const float* sa,
 /* ------------------------------------------------------------------ */
 
 /* The launch plan fp8_block_gemm uses for (M, N, K) on a device with `sms`
- * SMs (fp8_gemm_per_tensor, fp8_gemm_per_channel and the ue8m0 GEMM run
- * the same tiles, with one CTA where this plan has a CTA pair), with
+ * SMs (fp8_gemm_per_tensor and fp8_gemm_per_channel use the same plan; the
+ * ue8m0 GEMM runs one CTA where this plan has a CTA pair), with
  * the split-K partials (or those of a split last wave) limited to ws_cap
  * bytes (SIZE_MAX: no limit; fp8_block_gemm_noalloc plans with its
  * scratch size).  Host only: no device is touched, so it runs anywhere.
