@@ -229,8 +229,10 @@ def test_plan_tile_choice_by_m_and_n(cuda_lib):
         assert key(m, 7168) == ("normal", 256)
         assert key(m, 18432) == ("normal", 128)
     for m in (129, 256, 512):
-        for n in (2048, 7168, 18432):
+        for n in (2048, 7168, 16384):
             assert key(m, n) == ("normal", 256)
+        for n in (16385, 18432, 24576):
+            assert key(m, n) == ("pair", 256)
     for m in (513, 1024, 4096):
         for n in (2048, 7168, 18432):
             assert key(m, n) == ("pair", 256)
