@@ -13,6 +13,15 @@
 // held in registers as packed pairs (fma.rn.f32x2 in place).  kNumBuf TMEM buffers rotate so
 // the MMAs of the next K blocks overlap the promotion of this one.
 //
+// CTA pairs (PAIR): a cluster of two CTAs computes a 256 x BN tile with
+// cta_group::2 MMAs issued by the leader; each CTA loads its own 128 rows of
+// the P tile and half of the Q tile, and holds its 128 rows of every partial
+// in its own TMEM.  Both CTAs promote; the peer's promotion warps hand TMEM
+// buffers back by arriving on the leader's barriers.  With BN = 256 (TS) the
+// epilogue converts the tile to bf16 into shared memory and bulk-stores it
+// (cp.async.bulk.tensor), so the promotion warps return to the next tile's
+// partials without waiting for the global stores.
+//
 // Warp roles (one CTA per SM, persistent over work units):
 //   warpgroup 0   warp 0: TMA producer (P and Q tiles of one K block per
 //                 pipeline stage); warp 1: TMEM allocation and the single
@@ -20,13 +29,14 @@
 //                 scale-slot writer (scale mode 2), otherwise idle; warp 3
 //                 idle.  With several
 //                 promotion warpgroups warpgroup 0 hands registers to them
-//                 (setmaxnreg 48/224 or 56/216 for two, 32/160 for three).
+//                 (setmaxnreg 40/232 or 56/216 for two, 32/160 for three).
 //   warpgroups 1+ promotion / epilogue: thread = one TMEM lane (tile row)
 //                 and a slice of kCW accumulator columns (128 for 256-wide
 //                 tiles, else at most 64); warpgroup w-1 owns columns
 //                 [(w-1)*kCW, w*kCW).  A thread loads its slice in chunks
-//                 of at most 64 columns and releases the TMEM buffer as
-//                 soon as the last chunk has landed.
+//                 (48 + 80 columns for 128-column slices, else at most 64)
+//                 and releases the TMEM buffer as soon as the last chunk
+//                 has landed.
 //
 // Operand roles.  The MMA computes D[128 rows, BN cols] = P * Q^T with P and
 // Q K-major tiles in shared memory (128-byte swizzle).
