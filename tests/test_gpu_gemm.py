@@ -67,6 +67,8 @@ def sample_points(M, N, g, n_random=4096):
     # scale rows in 16-byte boxes (K/128 % 4 == 0): ragged M, N past the last
     # weight block, split-K ranges starting inside a group of 4 K blocks
     (300, 600, 2048), (520, 300, 512), (520, 640, 1536), (200, 1100, 3072),
+    # CTA-pair tiles (M > 512) with a single K block and with 128 K blocks
+    (600, 600, 128), (600, 520, 16384),
 ])
 def test_gemm_small_full(oracle_mod, gpu, m, n, k):
     qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=m * 131 + n * 7 + k)
