@@ -33,6 +33,7 @@ bool log_enabled() {
     return on;
 }
 
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 bool aligned8(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 7) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3) == 0; }
@@ -748,6 +749,22 @@ static int run_group128(const void* x, int64_t M, int64_t K, int64_t ldx, uint8_
     const int64_t G = K / 128, groups = M * G;
     constexpr int kGroupU = 2;        // groups per thread per iteration (8 threads a group)
     const bool contig = ldx == K && ldq == K;
+    if (contig && aligned32(x) && aligned16(q)) {
+        // 4 threads a group, 32-byte loads: 4-13 % faster than 8 threads a
+        // group at 1024-4096 x 7168 and 4000 x 1280, level at 16384 x 7168
+        constexpr int64_t kChunk = int64_t(kQuantThreads / 4);
+        const int64_t chunks = (groups + kChunk - 1) / kChunk;
+        const uint4* xv = static_cast<const uint4*>(x);
+        uint4* qv = reinterpret_cast<uint4*>(q);
+        const int grid = e8 ? chunk_grid<group128_contig4_kernel<true>>(chunks, d->sms)
+                            : chunk_grid<group128_contig4_kernel<false>>(chunks, d->sms);
+        if (log_enabled())
+            std::fprintf(stderr, "[fp8q] group128%s M=%lld K=%lld: 4 threads a group, grid=%d, %lld chunks\n",
+                         e8 ? " ue8m0" : "", (long long)M, (long long)K, grid, (long long)chunks);
+        if (e8) launch(group128_contig4_kernel<true>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xv, qv, scales, groups);
+        else launch(group128_contig4_kernel<false>, dim3(grid), dim3(kQuantThreads), 0, st, 1u, xv, qv, scales, groups);
+        return launch_status();
+    }
     if (contig) {
         constexpr int64_t kChunk = int64_t(kQuantThreads / 8) * kGroupU;
         const int64_t chunks = (groups + kChunk - 1) / kChunk;

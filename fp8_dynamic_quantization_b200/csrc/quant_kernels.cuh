@@ -6,11 +6,13 @@
 // dynamic-quant amax grid to the input", Description: a fixed 1024-block
 // grid with a 1024-way atomic sets a data-independent floor).
 //
-//  group128_contig_kernel /  one pass: amax of each 1x128 group, its scale,
-//  group128_quant_kernel     codes ("How to Profile DeepSeek-V3 Inference
-//                            Kernels Using Triton Autotuning", Benchmarking
+//  group128_contig4_kernel / one pass: amax of each 1x128 group, its scale,
+//  group128_contig_kernel /  codes ("How to Profile DeepSeek-V3 Inference
+//  group128_quant_kernel     Kernels Using Triton Autotuning", Benchmarking
 //                            the Activation Quantization Kernel); the first
-//                            for contiguous tensors, the second for strided.
+//                            for contiguous tensors with 32-byte aligned
+//                            input and 16-byte aligned codes, the second for
+//                            other contiguous tensors, the third for strided.
 //  amax_contig_kernel /      per-tensor amax, one partial max per CTA
 //  amax_partial_kernel       (contiguous / strided).
 //  apply_contig_kernel /     per-tensor apply pass (contiguous / strided):
@@ -323,6 +325,55 @@ group128_contig_kernel(const uint4* __restrict__ x, uint2* __restrict__ q, void*
                 if (sub == 0) static_cast<float*>(scales)[g] = d.s;
             }
         }
+    }
+}
+
+// Per-1x128-group quantisation of a contiguous [M, K] tensor with 4 threads
+// per group and 32-byte loads: thread `sub` of a group reads its vectors
+// 2sub, 2sub+1 and 8+2sub, 9+2sub (a warp's load covers 8 whole groups in
+// 128-byte runs) and stores its codes 16 bytes at a time.  A CTA takes 64
+// consecutive groups per iteration; a warp's 8 groups are in or out of range
+// together except in the last chunk.  x must be 32-byte aligned, q 16-byte.
+template <bool E8 = false>
+__global__ void __launch_bounds__(kQuantThreads)
+group128_contig4_kernel(const uint4* __restrict__ x, uint4* __restrict__ q, void* __restrict__ scales,
+                        int64_t groups) {
+    pdl_begin();
+    constexpr int kChunk = kQuantThreads / 4;               // groups per chunk (64)
+    const int sub = threadIdx.x & 3;
+    const int gl = threadIdx.x >> 2;                        // group within a chunk
+    const int64_t nchunks = (groups + kChunk - 1) / kChunk;
+    for (int64_t c = blockIdx.x; c < nchunks; c += gridDim.x) {
+        const int64_t g = c * kChunk + gl;
+        const bool full = c * kChunk + kChunk <= groups;
+        // a warp's eight groups: test the first, so the shuffles stay warp-uniform
+        if (!full && (g - (gl & 7)) >= groups) continue;
+        const bool ok = full || g < groups;
+        uint4 v[4];
+        if (ok) {
+            ld_stream32(x + g * 16 + 2 * sub, v[0], v[1]);  // a group is 16 vectors of 8 values
+            ld_stream32(x + g * 16 + 8 + 2 * sub, v[2], v[3]);
+        } else {
+            v[0] = v[1] = v[2] = v[3] = make_uint4(0, 0, 0, 0);
+        }
+        uint32_t m = max(max(absmax8(v[0]), absmax8(v[1])), max(absmax8(v[2]), absmax8(v[3])));
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+        m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+        if (!ok) continue;
+        uint2 c0, c1, c2, c3;
+        if (E8) {
+            const uint32_t sb = e8m0_from_amax_bits(m);
+            const float inv = e8m0_inverse(sb);
+            c0 = quant8_pow2(v[0], inv); c1 = quant8_pow2(v[1], inv);
+            c2 = quant8_pow2(v[2], inv); c3 = quant8_pow2(v[3], inv);
+            if (sub == 0) static_cast<uint8_t*>(scales)[g] = uint8_t(sb);
+        } else {
+            const Scale d = make_scale(scale_from_amax_bits(m));
+            c0 = quant8(v[0], d); c1 = quant8(v[1], d); c2 = quant8(v[2], d); c3 = quant8(v[3], d);
+            if (sub == 0) static_cast<float*>(scales)[g] = d.s;
+        }
+        st_stream16(q + g * 8 + sub, make_uint4(c0.x, c0.y, c1.x, c1.y));      // codes: 8 vectors of 16
+        st_stream16(q + g * 8 + 4 + sub, make_uint4(c2.x, c2.y, c3.x, c3.y));
     }
 }
 

@@ -77,6 +77,37 @@ def test_group128_strided_rows(oracle_mod, gpu):
     assert_codes_equal(_u8(q), q_ref)
 
 
+# Contiguous tensors take the 4-threads-a-group kernel when x is 32-byte and
+# the codes 16-byte aligned, the 8-threads-a-group kernel otherwise: each
+# alignment pair is run through the C ABI with buffers placed at that offset.
+@pytest.mark.parametrize("x_off,q_off", [(0, 0), (16, 0), (0, 8), (48, 24)])
+@pytest.mark.parametrize("m,k", [(33, 1280), (1000, 7168)])
+@pytest.mark.parametrize("e8", [False, True])
+def test_group128_contiguous_alignments(oracle_mod, gpu, x_off, q_off, m, k, e8):
+    lib = fq.library()
+    x = inputs.activations_group(m, k=k, seed=m + k + x_off)
+    if e8:
+        q_ref, s_ref = oracle_mod.quant_group128_ue8m0(inputs.bf16_bits(x))
+    else:
+        q_ref, s_ref = oracle_mod.quant_group128(inputs.bf16_bits(x))
+    xb = torch.empty(m * k * 2 + 64, dtype=torch.uint8, device=gpu)
+    xb[x_off:x_off + m * k * 2].copy_(x.to(gpu).view(torch.uint8).reshape(-1))
+    qb = torch.empty(m * k + 64, dtype=torch.uint8, device=gpu)
+    g = k // 128
+    s = torch.empty(m * g, dtype=torch.uint8 if e8 else torch.float32, device=gpu)
+    st = torch.cuda.current_stream().cuda_stream
+    fn = lib.fp8_act_quant_group128_ue8m0 if e8 else lib.fp8_act_quant_group128
+    assert fn(xb.data_ptr() + x_off, m, k, k, qb.data_ptr() + q_off, k, s.data_ptr(), st) == 0
+    torch.cuda.synchronize()
+    q = qb[q_off:q_off + m * k].reshape(m, k).cpu().numpy()
+    if e8:
+        assert np.array_equal(s.cpu().numpy().reshape(m, g), s_ref.reshape(m, g))
+    else:
+        assert_scales_equal(s.cpu().numpy().reshape(m, g), s_ref)
+    assert_codes_equal(q, q_ref)
+    assert fq.device_status() == 0
+
+
 def test_group128_zero_groups_and_signed_zeros(oracle_mod, gpu):
     x = inputs.activations_group(6, k=512, seed=2)
     x[1, 128:256] = 0.0
