@@ -1,7 +1,8 @@
 // Quantisation kernels: bf16 -> E4M3 codes + fp32 scales (sm_100a).
 //
 // All of them are HBM-bound streaming kernels: 16-byte vector loads of 8
-// bf16 values, several loads in flight per thread, grids sized to the input
+// bf16 values (32-byte loads in group128_contig4_kernel), several loads in
+// flight per thread, grids sized to the input
 // (never a fixed grid with idle blocks; compare "Size the per-tensor FP8
 // dynamic-quant amax grid to the input", Description: a fixed 1024-block
 // grid with a 1024-way atomic sets a data-independent floor).
