@@ -8,7 +8,7 @@ every canary byte must be intact and the output must equal the same call
 made into a plain buffer.  Two canary values are used, so a stray write of
 one of them is still caught by the other run.  Shapes are ragged (rows and
 columns off the tile sizes, short last chunks) and cover the chunked and
-strided quantisation kernels, the CTA-pair GEMM with its bulk-store
+strided quantisation kernels (fp32 and ue8m0 group scales), the CTA-pair GEMM with its bulk-store
 epilogue and split last wave, the single-CTA tiles and the swapped split-K
 path.  Calls go through the C ABI with these buffers (ctypes)."""
 import numpy as np
@@ -80,21 +80,28 @@ def test_per_tensor_quant_writes_only_its_outputs(gpu, m, k, ldq):
     assert fq.device_status() == 0
 
 
-@pytest.mark.parametrize("m,k,ldq", [(4096, 7168, 7168), (1000, 1280, 1280), (97, 2048, 2048 + 128)])
-def test_group128_quant_writes_only_its_outputs(gpu, m, k, ldq):
+@pytest.mark.parametrize("m,k,ldq", [(4096, 7168, 7168), (1000, 1280, 1280), (129, 7168, 7168),
+                                     (97, 2048, 2048 + 128)])
+@pytest.mark.parametrize("e8", [False, True])
+def test_group128_quant_writes_only_its_outputs(gpu, m, k, ldq, e8):
     lib = _lib()
     x = inputs.activations_group(m, k=k, seed=m + k).to(gpu)
-    q_ref, s_ref = fq.act_quant_group128(x)
+    q_ref, s_ref = fq.act_quant_group128_ue8m0(x) if e8 else fq.act_quant_group128(x)
     g = k // 128
+    fn = lib.fp8_act_quant_group128_ue8m0 if e8 else lib.fp8_act_quant_group128
     for canary in CANARIES:
         q = Guarded(gpu, m, k, ldq, 1, canary)
-        s = Guarded(gpu, m, g, g, 4, canary)
-        assert lib.fp8_act_quant_group128(x.data_ptr(), m, k, k, q.ptr(), ldq, s.ptr(), _stream()) == 0
+        s = Guarded(gpu, m, g, g, 1 if e8 else 4, canary)
+        assert fn(x.data_ptr(), m, k, k, q.ptr(), ldq, s.ptr(), _stream()) == 0
         torch.cuda.synchronize()
         q.check("group codes")
         s.check("group scales")
         assert torch.equal(q.output(), q_ref.view(torch.uint8))
-        assert torch.equal(s.output().contiguous().view(torch.float32).reshape(m, g), s_ref)
+        got = s.output().contiguous()
+        if e8:
+            assert torch.equal(got.reshape(m, g), s_ref.view(torch.uint8).reshape(m, g))
+        else:
+            assert torch.equal(got.view(torch.float32).reshape(m, g), s_ref)
     assert fq.device_status() == 0
 
 
