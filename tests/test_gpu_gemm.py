@@ -78,6 +78,23 @@ def test_gemm_small_full(oracle_mod, gpu, m, n, k):
     assert fq.device_status() == 0
 
 
+# Seeded random shapes (N a multiple of 8 for the 16-byte row pitch of Y):
+# M up to 1099 and N up to 1272 reach the swapped, single-CTA and CTA-pair
+# rows of the launch table, with ragged tiles in both dimensions and a
+# range of split-K and split-tail counts.
+def test_gemm_random_shapes(oracle_mod, gpu):
+    g = np.random.default_rng(2468)
+    for case in range(16):
+        m = int(g.integers(1, 1100))
+        n = 8 * int(g.integers(1, 160))
+        k = 128 * int(g.integers(1, 13))
+        qa, sa, qb, sb = inputs.gemm_operands(m, n, k, seed=11000 + case)
+        y = run_gemm(qa, sa, qb, sb, gpu)
+        R, T = oracle_mod.block_gemm(qa, sa, qb, sb)
+        assert_within(oracle_mod, y_f64(y), R, T, f"random {m}x{n}x{k}")
+    assert fq.device_status() == 0
+
+
 @pytest.mark.parametrize("m", [1, 16, 64, 256])
 @pytest.mark.parametrize("n", [2048, 7168, 18432])
 def test_gemm_decode_shapes(oracle_mod, gpu, m, n):

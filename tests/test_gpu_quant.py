@@ -108,6 +108,28 @@ def test_group128_contiguous_alignments(oracle_mod, gpu, x_off, q_off, m, k, e8)
     assert fq.device_status() == 0
 
 
+# Seeded random shapes: row counts that leave every possible ragged last
+# chunk of the 64-group and 32-group kernels, K from one group to 16, fp32
+# and ue8m0 scales, each through the Python binding (aligned buffers).
+def test_group128_random_shapes(oracle_mod, gpu):
+    g = np.random.default_rng(1234)
+    for case in range(24):
+        m = int(g.integers(1, 400))
+        k = 128 * int(g.integers(1, 17))
+        x = inputs.activations_group(m, k=k, seed=7000 + case, dist="normal" if case % 2 else "laplace")
+        bits = inputs.bf16_bits(x)
+        if case % 3 == 0:
+            q, s = fq.act_quant_group128_ue8m0(x.to(gpu))
+            q_ref, s_ref = oracle_mod.quant_group128_ue8m0(bits)
+            assert np.array_equal(s.cpu().numpy(), np.asarray(s_ref).reshape(m, k // 128)), (m, k)
+        else:
+            q, s = fq.act_quant_group128(x.to(gpu))
+            q_ref, s_ref = oracle_mod.quant_group128(bits)
+            assert_scales_equal(s.cpu().numpy(), s_ref)
+        assert_codes_equal(_u8(q), q_ref)
+    assert fq.device_status() == 0
+
+
 def test_group128_zero_groups_and_signed_zeros(oracle_mod, gpu):
     x = inputs.activations_group(6, k=512, seed=2)
     x[1, 128:256] = 0.0
@@ -155,6 +177,21 @@ def test_per_tensor_other_shapes(oracle_mod, gpu, m, k):
     q, s = fq.act_quant_per_tensor(x.to(gpu))
     assert_scales_equal(s.cpu().numpy(), np.array([s_ref]))
     assert_codes_equal(_u8(q), q_ref)
+
+
+# Seeded random shapes across the one-cluster path (small tensors), the
+# half-size and full-size amax chunks, and ragged last chunks.
+def test_per_tensor_random_shapes(oracle_mod, gpu):
+    g = np.random.default_rng(4321)
+    for case in range(20):
+        m = int(g.integers(1, 3000))
+        k = 8 * int(g.integers(1, 400))
+        x = inputs.activations_per_tensor(m, k=k, seed=9000 + case)
+        q_ref, s_ref = oracle_mod.quant_per_tensor(inputs.bf16_bits(x))
+        q, s = fq.act_quant_per_tensor(x.to(gpu))
+        assert_scales_equal(s.cpu().numpy(), np.array([s_ref]))
+        assert_codes_equal(_u8(q), q_ref)
+    assert fq.device_status() == 0
 
 
 def test_per_tensor_repeated_calls_reuse_workspace(oracle_mod, gpu):
