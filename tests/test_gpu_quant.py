@@ -305,3 +305,22 @@ def test_every_x_and_amax_pair(oracle_mod, gpu):
                     s_np[i].view(np.uint32) == np.float32(s_ref).view(np.uint32)):
                 assert_scales_equal(s_np[i:i + 1], np.array([s_ref]))
                 assert_codes_equal(got_np[i], want)
+
+
+def test_empty_inputs_every_quant_entry_point(gpu):
+    """Zero rows (and, for the GEMM-side scales, zero weight rows) give empty
+    outputs of the right shapes, enqueue nothing that faults, and leave no
+    device error."""
+    for k in (128, 7168):
+        x = torch.empty(0, k, dtype=torch.bfloat16, device=gpu)
+        q, s = fq.act_quant_group128(x)
+        assert q.shape == (0, k) and s.shape == (0, k // 128)
+        q, s = fq.act_quant_group128_ue8m0(x)
+        assert q.shape == (0, k) and s.shape == (0, k // 128)
+        q, s = fq.act_quant_per_channel(x)
+        assert q.shape == (0, k) and s.numel() == 0
+        q, s = fq.weight_quant_block128(x)
+        assert q.shape == (0, k) and s.numel() == 0
+        q, s = fq.weight_quant_block128_ue8m0(x)
+        assert q.shape == (0, k) and s.numel() == 0
+    assert fq.device_status() == 0
