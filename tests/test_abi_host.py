@@ -6,6 +6,8 @@ import os
 import re
 
 import pytest
+from hypothesis import given, settings
+from hypothesis import strategies as st
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "fp8q.h")
@@ -271,3 +273,44 @@ def test_plan_depends_on_the_sm_count(cuda_lib):
     # 4096 x 7168 on 132 SMs (66 pairs): 448 = 6 * 66 + 52 -> more than half a wave
     p = gemm_plan(cuda_lib, 4096, 7168, 7168, sms=132)
     assert (p["tail_tiles"], p["grid"]) == (0, 132)
+
+
+@settings(max_examples=400, deadline=None)
+@given(m=st.one_of(st.integers(1, 40), st.integers(1, 600), st.integers(1, 20000)),
+       n=st.one_of(st.integers(1, 2100), st.integers(1, 40000)), g=st.integers(1, 128),
+       sms=st.integers(4, 80).map(lambda h: 2 * h), capped=st.booleans())
+def test_plan_invariants(cuda_lib, m, n, g, sms, capped):
+    """Whatever the shape, SM count and workspace cap: the tiles cover the
+    output, every work unit has at least one K block, the grid fits the SMs
+    (an even count for CTA pairs), and the workspace is what the partials
+    need (within the cap unless the swapped minimum of two K ranges is
+    forced)."""
+    k = 128 * g
+    cap = NOALLOC_CAP if capped else NO_CAP
+    p = gemm_plan(cuda_lib, m, n, k, sms=sms, cap=cap)
+    rows = 256 if p["pair"] else 128
+    if p["swap"]:
+        assert not p["pair"] and p["bn"] <= 128
+        assert p["tiles_p"] == -(-n // 128) and p["tiles_q"] == -(-m // p["bn"])
+    else:
+        assert p["tiles_p"] == -(-m // rows) and p["tiles_q"] == -(-n // p["bn"])
+    tiles = p["tiles_p"] * p["tiles_q"]
+    assert 1 <= p["splits"] <= g
+    if p["tail_tiles"]:
+        slots = sms // 2 if p["pair"] else sms
+        assert p["splits"] == 1 and not p["swap"]
+        assert tiles > slots and p["tail_tiles"] == tiles % slots
+        assert 2 <= p["tail_splits"] <= min(slots // p["tail_tiles"], g // 2)
+        assert p["units"] == tiles - p["tail_tiles"] + p["tail_tiles"] * p["tail_splits"]
+        assert p["ws"] == p["tail_tiles"] * p["tail_splits"] * rows * p["bn"] * 4
+    else:
+        assert p["tail_splits"] == 1 and p["units"] == tiles * p["splits"]
+        ldw = -(-n // 8) * 8
+        assert p["ws"] == (p["splits"] * m * ldw * 4 if p["splits"] > 1 else 0)
+    if p["pair"]:
+        assert p["grid"] % 2 == 0 and p["grid"] == 2 * max(1, min(p["units"], sms // 2))
+    else:
+        assert p["grid"] == max(1, min(p["units"], sms))
+    # the swapped kernel takes at most 64 K blocks per unit, cap or not
+    forced = p["swap"] and g > 64 and p["splits"] == -(-g // 64)
+    assert p["ws"] <= cap or forced
